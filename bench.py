@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the W2A8 BitLinear hot path on B200.
+
+Headline workload: the W2A8 GEMV shape sweep at M = 1 (eight (N, K) shapes,
+uniform int8 activations in [-127, 127], ternary weights with P = 1/3 each,
+int32 output).  One step = one pass over the eight shapes, each through
+bitnet_w2a8_gemm.  Metric: achieved HBM GB/s with algorithmic bytes
+N*K/4 + M*K + 4*M*N per call; per-shape us/call are in "details".
+Extra lines of "details": the large GEMV shapes, the BitLinear decode
+(M = 1, bf16 in/out) and the prefill GEMM int8 TOPS (M >= 128).
+
+Timing: inputs resident in HBM; the weights rotate over enough copies that
+each step's set was last read more than 2x L2 capacity ago (no L2 reuse
+between steps); each step is one CUDA-graph replay; CUDA events on the
+launching stream; max over ranks.  `--impl reference` times the CPU oracle
+instead (rank 0 only).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ternary_weight_bit_w2a8_b200 import synth  # noqa: E402
+
+METRIC = "W2A8 GEMV us/call & HBM GB/s (% of peak) at M=1; int8 TOPS at M=128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES_DEFAULT = 126 * 2**20
+
+
+def gemv_bytes(M, N, K):
+    """Algorithmic bytes of one call: packed weights + int8 activations + int32 outputs."""
+    return N * K / 4 + M * K + 4 * M * N
+
+
+def bitlinear_bytes(M, N, K):
+    return N * K / 4 + 2 * M * K + 2 * M * N
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while it runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, period_ms: int = 50):
+        self.gpu_id = gpu_id
+        self.period_ms = period_ms
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(2 * self.period_ms / 1000)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(torch, dev):
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return "GPU-" + str(p.uuid)
+    except Exception:
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+
+
+# ----------------------------------------------------------------------------- helpers
+def to_dev(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def bf16_dev(torch, bits):
+    return to_dev(torch, bits.view(np.int16)).view(torch.bfloat16)
+
+
+def timed_graph_loop(torch, graphs, steps, warmup, dist=None):
+    """Replays graphs round-robin: `warmup` untimed, then exactly `steps` timed.
+    Returns the elapsed ms (max over ranks)."""
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+def capture(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the library (device info, function attributes) outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def rotation_copies(total_bytes, l2_bytes):
+    return max(3, int(math.ceil(2 * l2_bytes / max(total_bytes, 1))) + 1)
+
+
+# ----------------------------------------------------------------------------- our arm
+class GemvSet:
+    """Device buffers for a list of M=1 GEMV shapes with rotating weight copies."""
+
+    def __init__(self, torch, bn, shapes, gen, seed, l2_bytes, max_copies=None):
+        self.torch, self.bn, self.shapes = torch, bn, shapes
+        self.q, self.y, self.ws, self.packed0 = [], [], [], []
+        total = 0
+        for (N, K) in shapes:
+            q, w = gen(N, K, seed=seed)
+            self.q.append(to_dev(torch, q))
+            self.packed0.append(bn.bitnet_pack_weights(to_dev(torch, w)))
+            del w
+            self.y.append(torch.empty((1, N), dtype=torch.int32, device="cuda"))
+            self.ws.append(bn.workspace(1, N, K))
+            total += bn.bitnet_packed_bytes(N, K)
+        c = rotation_copies(total, l2_bytes)
+        if max_copies:
+            c = min(c, max_copies)
+        self.copies = [self.packed0] + [[p.clone() for p in self.packed0] for _ in range(c - 1)]
+        self.packed_total = total
+        self.bytes_per_step = sum(gemv_bytes(1, N, K) for N, K in shapes)
+        torch.cuda.synchronize()
+
+    def run(self, c, events=None):
+        for j, (N, K) in enumerate(self.shapes):
+            if events is not None:
+                events[j][0].record()
+            self.bn.bitnet_w2a8_gemm(self.q[j], self.copies[c][j], N, y=self.y[j], ws=self.ws[j])
+            if events is not None:
+                events[j][1].record()
+
+
+def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
+    """Graph per rotation copy (one step each, timing events around each call)."""
+    torch = gs.torch
+    evs, graphs = [], []
+    n_before = bn.bitnet_launch_count()
+    for c in range(len(gs.copies)):
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in gs.shapes]
+        graphs.append(capture(torch, lambda c=c, ev=ev: gs.run(c, ev)))
+        evs.append(ev)
+    launches_per_step = (bn.bitnet_launch_count() - n_before) // (2 * len(gs.copies))
+    if clocks is not None:
+        clocks.start()
+    ms = timed_graph_loop(torch, graphs, steps, warmup, dist)
+    clk = clocks.stop() if clocks is not None else None
+    # per-launch durations: the last replay of every graph
+    per_shape_us = []
+    for j in range(len(gs.shapes)):
+        d = [evs[c][j][0].elapsed_time(evs[c][j][1]) * 1e3 for c in range(len(gs.copies))]
+        per_shape_us.append(float(np.mean(d)))
+    del graphs
+    return ms, per_shape_us, launches_per_step, clk
+
+
+def e2e_sweep(torch, bn, gs, steps):
+    """Through the public API with host buffers: pinned activations -> device,
+    the call, device -> pinned int32 result, synchronised every step."""
+    hq = [q.cpu().pin_memory() for q in gs.q]
+    hy = [torch.empty(y.shape, dtype=torch.int32).pin_memory() for y in gs.y]
+    h2d = sum(q.numel() for q in hq)
+    d2h = sum(y.numel() * 4 for y in hy)
+    for i in range(3):
+        for j, (N, K) in enumerate(gs.shapes):
+            gs.q[j].copy_(hq[j], non_blocking=True)
+            bn.bitnet_w2a8_gemm(gs.q[j], gs.copies[i % len(gs.copies)][j], N, y=gs.y[j], ws=gs.ws[j])
+            hy[j].copy_(gs.y[j], non_blocking=True)
+        torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        for j, (N, K) in enumerate(gs.shapes):
+            gs.q[j].copy_(hq[j], non_blocking=True)
+            bn.bitnet_w2a8_gemm(gs.q[j], gs.copies[i % len(gs.copies)][j], N, y=gs.y[j], ws=gs.ws[j])
+            hy[j].copy_(gs.y[j], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    return ms, h2d, d2h
+
+
+def measure_bitlinear_decode(torch, bn, shapes, steps, warmup, l2_bytes):
+    out = []
+    for (N, K) in shapes:
+        x, W = synth.bitlinear_inputs(1, N, K, seed=0)
+        Wd = bf16_dev(torch, W)
+        gamma = bn.bitnet_absmean(Wd)
+        packed = bn.bitnet_pack_weights(bn.bitnet_ternarize(Wd, gamma))
+        del Wd
+        c = rotation_copies(packed.numel(), l2_bytes)
+        copies = [packed] + [packed.clone() for _ in range(c - 1)]
+        xd = bf16_dev(torch, x)
+        y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+        ws = bn.workspace(1, N, K)
+        graphs = [capture(torch, lambda p=p: bn.bitnet_bitlinear(xd, p, gamma, N, y=y, ws=ws)) for p in copies]
+        ms = timed_graph_loop(torch, graphs, steps, warmup)
+        us = ms * 1e3 / steps
+        out.append({"N": N, "K": K, "us_per_call": round(us, 3),
+                    "GBps": round(bitlinear_bytes(1, N, K) / (us * 1e-6) / 1e9, 1)})
+        del graphs, copies
+    return out
+
+
+def measure_prefill(torch, bn, ms_list, shapes, steps, warmup, int8_peak_tops):
+    out = []
+    for (N, K) in shapes:
+        W = synth.bf16_weights(N, K, seed=1)
+        Wd = bf16_dev(torch, W)
+        gamma = bn.bitnet_absmean(Wd)
+        packed = bn.bitnet_pack_weights(bn.bitnet_ternarize(Wd, gamma))
+        del Wd
+        for M in ms_list:
+            x = synth.bf16_activations(M, K, seed=0, outlier_p=0.0)
+            xd = bf16_dev(torch, x)
+            q, s, _ = bn.bitnet_quant_act(xd)
+            y = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            ws = bn.workspace(M, N, K)
+            g = capture(torch, lambda: bn.bitnet_w2a8_gemm(q, packed, N, y=y, ws=ws))
+            n = max(3, steps)
+            ms = timed_graph_loop(torch, [g], n, warmup)
+            us = ms * 1e3 / n
+            tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            out.append({"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "int8_TOPS": round(tops, 1),
+                        "frac_int8_peak": round(tops / int8_peak_tops, 4),
+                        "GBps": round(gemv_bytes(M, N, K) / (us * 1e-6) / 1e9, 1)})
+            del g
+    return out
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import ternary_weight_bit_w2a8_b200 as bn
+    from ternary_weight_bit_w2a8_b200 import build
+    if rank == 0 or not os.path.exists(bn.LIB_PATH):
+        build.build()
+    if dist is not None:
+        dist.barrier()
+    dev = torch.cuda.current_device()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_DEFAULT
+    peaks = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    int8_peak = 2.0 * float(peaks["bf16_tflops"])  # dense int8 = 2x dense bf16 (nominal ratio)
+
+    gs = GemvSet(torch, bn, synth.SWEEP_SHAPES, synth.uniform_int8_ternary, seed=rank, l2_bytes=l2)
+    clocks = ClockSampler(gpu_id_for(torch, dev)) if rank == 0 else None
+    ms, per_shape_us, launches_per_step, clk = measure_gemv_set(torch, bn, gs, args.steps, args.warmup, dist,
+                                                                clocks)
+    ms_per_step = ms / args.steps
+    value = world * gs.bytes_per_step * args.steps / (ms * 1e-3) / 1e9
+    kern_us = sum(per_shape_us)
+    achieved = gs.bytes_per_step / (kern_us * 1e-6) / 1e9
+
+    e2e_steps = max(3, min(args.steps, 300))
+    e2e_ms, h2d, d2h = e2e_sweep(torch, bn, gs, e2e_steps)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * gs.bytes_per_step * e2e_steps / (e2e_ms * 1e-3) / 1e9
+
+    details = {"sweep": [{"N": N, "K": K, "us_per_call": round(u, 3),
+                          "GBps": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9, 1),
+                          "frac_hbm": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9 / hbm_peak, 4)}
+                         for (N, K), u in zip(synth.SWEEP_SHAPES, per_shape_us)]}
+    del gs
+    torch.cuda.empty_cache()
+    if not args.quick and rank == 0:
+        gl = GemvSet(torch, bn, synth.LARGE_SHAPES, synth.sparse_ternary_normal_int8, seed=0, l2_bytes=l2)
+        n = max(20, min(args.steps, 2000))
+        _, us_l, _, _ = measure_gemv_set(torch, bn, gl, n, max(3, args.warmup))
+        details["large"] = [{"N": N, "K": K, "us_per_call": round(u, 3),
+                             "GBps": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9, 1),
+                             "frac_hbm": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9 / hbm_peak, 4)}
+                            for (N, K), u in zip(synth.LARGE_SHAPES, us_l)]
+        del gl
+        torch.cuda.empty_cache()
+        details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
+                                                               max(20, min(args.steps, 2000)), max(3, args.warmup), l2)
+        details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES,
+                                             max(10, min(args.steps // 20, 200)), max(3, args.warmup), int8_peak)
+        details["int8_peak_tops"] = {"value": round(int8_peak, 1),
+                                     "basis": f"{peaks['source']} bf16 dense x 2 (nominal int8/bf16 ratio)"}
+
+    err = bn.bitnet_get_device_error()
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8xint2->int32", "data": "synthetic",
+        "config": {"workload": "W2A8 GEMV M=1 shape sweep, 8 (N,K) shapes, int32 out",
+                   "shapes": [list(s) for s in synth.SWEEP_SHAPES],
+                   "l2": f"weights rotate over {len(synth.SWEEP_SHAPES)}-shape sets, "
+                         f"{rotation_copies(sum(N * K // 4 for N, K in synth.SWEEP_SHAPES), l2)} copies "
+                         f"(> 2x L2 of {l2 // 2**20} MiB between reuses)",
+                   "step": "one CUDA-graph replay of the 8 bitnet_w2a8_gemm calls",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "seed": "rank"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "kernel": "gemv_w2a8_kernel", "peak_source": peaks["source"],
+                     "per_launch_bytes": "N*K/4 + K + 4N per shape, mean over the 8 shapes"},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps,
+                "note": "public API calls with pinned host activations copied in and int32 results copied out "
+                        "every step, stream synchronised per step; packed weights resident"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "device_error": err,
+        "details": details,
+    }
+
+
+# ----------------------------------------------------------------------------- CPU arms
+def oracle_sweep_step(shapes_data, frac, step):
+    """One oracle pass over a row sample of every sweep shape; returns algorithmic bytes processed."""
+    import oracle
+    done = 0.0
+    for (q, w, N, K) in shapes_data:
+        rows = max(1, int(N * frac))
+        r0 = (step * rows) % N
+        first = min(rows, N - r0)
+        oracle.gemm_i32(q, w[r0:r0 + first])  # contiguous row blocks: no copy
+        if first < rows:
+            oracle.gemm_i32(q, w[:rows - first])
+        done += gemv_bytes(1, rows, K)
+    return done
+
+
+def cpu_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def cpu_baseline(budget_s=4.0):
+    """The oracle, as it stands, on a bounded row sample of the sweep."""
+    import oracle
+    oracle._lib()
+    data = []
+    for (N, K) in synth.SWEEP_SHAPES:
+        q, w = synth.uniform_int8_ternary(N, K, seed=0)
+        data.append((q, w, N, K))
+    frac = 1.0 / 16
+    t0 = time.perf_counter()
+    oracle_sweep_step(data, frac, 0)
+    t1 = time.perf_counter()
+    reps = max(1, int(budget_s / max(t1 - t0, 1e-6)))
+    done = 0.0
+    t0 = time.perf_counter()
+    for i in range(reps):
+        done += oracle_sweep_step(data, frac, i + 1)
+    dt = time.perf_counter() - t0
+    return {"value": round(done / dt / 1e9, 3), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{reps} passes over 1/16 of the rows of each of the 8 sweep shapes "
+                      f"(algorithmic bytes of the rows processed), {dt:.1f} s"}
+
+
+def run_reference(args):
+    import oracle
+    oracle._lib()
+    data = []
+    for (N, K) in synth.SWEEP_SHAPES:
+        q, w = synth.uniform_int8_ternary(N, K, seed=0)
+        data.append((q, w, N, K))
+    t0 = time.perf_counter()
+    oracle_sweep_step(data, 1.0 / 64, 0)
+    t_probe = (time.perf_counter() - t0) * 64  # seconds for one full sweep
+    budget = 90.0 / max(1, args.steps + args.warmup)  # whole run within ~1.5 min
+    frac = min(1.0, budget / max(t_probe, 1e-9))
+    for i in range(args.warmup):
+        oracle_sweep_step(data, frac, i)
+    done = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        done += oracle_sweep_step(data, frac, args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = done / dt / 1e9
+    sample = f"each step: {frac:.3g} of the rows of each of the 8 sweep shapes"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8xint2->int32",
+            "data": "synthetic",
+            "config": {"workload": "W2A8 GEMV M=1 shape sweep, 8 (N,K) shapes, int32 out",
+                       "shapes": [list(s) for s in synth.SWEEP_SHAPES]},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle", "cores": cpu_threads(),
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline only (skip the details workloads)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    try:
+        res = run_ours(args, rank, world, dist)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
