@@ -210,25 +210,38 @@ class GemvSet:
 
 
 def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
-    """Graph per rotation copy (one step each, timing events around each call)."""
+    """Headline: one event-free graph per rotation copy (one step each, so
+    programmatic dependent launch links the calls), replayed round-robin.
+    Per-launch durations: a second timed loop over graphs with timing events
+    around every call (events between calls also break the launch overlap, so
+    these durations are conservative)."""
     torch = gs.torch
-    evs, graphs = [], []
     n_before = bn.bitnet_launch_count()
-    for c in range(len(gs.copies)):
-        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in gs.shapes]
-        graphs.append(capture(torch, lambda c=c, ev=ev: gs.run(c, ev)))
-        evs.append(ev)
+    graphs = [capture(torch, lambda c=c: gs.run(c)) for c in range(len(gs.copies))]
     launches_per_step = (bn.bitnet_launch_count() - n_before) // (2 * len(gs.copies))
     if clocks is not None:
         clocks.start()
     ms = timed_graph_loop(torch, graphs, steps, warmup, dist)
     clk = clocks.stop() if clocks is not None else None
-    # per-launch durations: the last replay of every graph
-    per_shape_us = []
-    for j in range(len(gs.shapes)):
-        d = [evs[c][j][0].elapsed_time(evs[c][j][1]) * 1e3 for c in range(len(gs.copies))]
-        per_shape_us.append(float(np.mean(d)))
     del graphs
+    evs, egraphs = [], []
+    for c in range(len(gs.copies)):
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in gs.shapes]
+        egraphs.append(capture(torch, lambda c=c, ev=ev: gs.run(c, ev)))
+        evs.append(ev)
+    n_ev = max(len(gs.copies), min(steps, 20 * len(gs.copies)))
+    per_shape = [[] for _ in gs.shapes]
+    for i in range(n_ev):
+        c = i % len(gs.copies)
+        egraphs[c].replay()
+        if c == len(gs.copies) - 1:
+            torch.cuda.synchronize()
+            for cc in range(len(gs.copies)):
+                for j in range(len(gs.shapes)):
+                    per_shape[j].append(evs[cc][j][0].elapsed_time(evs[cc][j][1]) * 1e3)
+    torch.cuda.synchronize()
+    per_shape_us = [float(np.mean(d)) if d else float("nan") for d in per_shape]
+    del egraphs
     return ms, per_shape_us, launches_per_step, clk
 
 
@@ -467,6 +480,28 @@ def run_reference(args):
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile(args):
+    """One problem, `steps` plain calls over rotating weight copies, no graphs."""
+    import torch
+    import ternary_weight_bit_w2a8_b200 as bn
+    M, N, K = (int(v) for v in args.profile.split(","))
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    gen = synth.sparse_ternary_normal_int8 if (N, K) in synth.LARGE_SHAPES else synth.uniform_int8_ternary
+    q, w = gen(N, K, seed=0, M=M)
+    qd = to_dev(torch, q)
+    packed = bn.bitnet_pack_weights(to_dev(torch, w))
+    del w
+    copies = [packed] + [packed.clone() for _ in range(rotation_copies(packed.numel(), l2) - 1)]
+    y = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    ws = bn.workspace(M, N, K)
+    for i in range(args.warmup + args.steps):
+        bn.bitnet_w2a8_gemm(qd, copies[i % len(copies)], N, y=y, ws=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": [M, N, K], "calls": args.warmup + args.steps,
+                      "device_error": bn.bitnet_get_device_error()}))
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -476,6 +511,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline only (skip the details workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", metavar="M,N,K",
+                    help="profiling mode: only `steps` plain bitnet_w2a8_gemm calls on one problem (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -489,6 +526,9 @@ def main():
             return 0
         print(json.dumps(run_reference(args)), flush=True)
         return 0
+
+    if args.profile:
+        return run_profile(args)
 
     import torch
     if not torch.cuda.is_available():

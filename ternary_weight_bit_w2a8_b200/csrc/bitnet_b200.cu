@@ -3,6 +3,8 @@
 // All kernels are in the headers included below; this is the library's single
 // translation unit, so file-scope device state (the error word) is shared.
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -17,13 +19,22 @@ std::atomic<int64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSliceChunks = 1536;  // activations of one K-slice: 96 KB of shared memory
-constexpr int kPlanSlots = 148 * 16;   // warp slots the GEMV plan aims to fill (fixed: plans depend on shape only)
+constexpr int kPlanSlots = 148 * 16;   // warp slots the K-split aims to fill (fixed: it sizes the workspace)
+constexpr int kOccCache = 128;
+
+struct OccEntry {
+    int idx;
+    size_t smem;
+    int ctas;
+};
 
 struct DeviceInfo {
     bool init = false;
     int status = BITNET_OK;
     int sm_count = 0;
     unsigned smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
+    int n_occ = 0;
+    OccEntry occ[kOccCache];     // resident CTAs per SM by (instantiation, shared memory)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -68,6 +79,21 @@ inline int grid_for(int64_t work, int64_t per_cta, int sm_count, int per_sm = 8)
     return (int)(g < 1 ? 1 : g);
 }
 
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ------------------------------------------------------------------ fill (K == 0)
 template <typename T>
 __global__ void __launch_bounds__(kThreads) fill_kernel(T *p, int64_t n, T v) {
@@ -75,104 +101,149 @@ __global__ void __launch_bounds__(kThreads) fill_kernel(T *p, int64_t n, T v) {
 }
 
 // ------------------------------------------------------------------ GEMV plan
-struct GemvPlan {
-    int G, R, UN, S, cps;
-    size_t smem;
+// The K-split depends on the shape only (it sizes the workspace); rows per
+// lane group and the grid also depend on the device.
+struct GemvSplit {
+    int S, cps;
     int64_t ws_bytes;
 };
 
-GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K) {
-    GemvPlan p{};
+inline int lanes_per_row(int nch) { return nch >= 128 ? 32 : (nch >= 48 ? 16 : 8); }
+
+GemvSplit plan_split(int64_t M, int64_t N, int64_t K) {
+    GemvSplit p{};
     const int nch = (int)(k_pad(K) / 64);
-    p.G = nch >= 128 ? 32 : (nch >= 48 ? 16 : 8);
-    const int64_t lanes_rows = 32 / p.G;
-    auto tasks = [&](int R) { return ceil_div(N, lanes_rows * R) * M; };
-    p.R = tasks(4) >= 2 * kPlanSlots ? 4 : (tasks(2) >= 2 * kPlanSlots ? 2 : 1);
+    const int G = lanes_per_row(nch);
+    const int64_t tasks = ceil_div(N, 32 / G) * M;  // warp tasks at one row per lane group
     int S = (int)ceil_div(nch, kMaxSliceChunks);
     // split K only when rows are too few to fill the GPU and every lane still
     // keeps >= 4 chunks per slice (small problems are latency-bound: a second
     // launch would cost more than it saves)
-    while (tasks(p.R) * S < kPlanSlots / 4 && nch / (2 * S) >= 4 * p.G) S *= 2;
+    while (tasks * S < kPlanSlots / 4 && nch / (2 * S) >= 4 * G) S *= 2;
     p.cps = (int)ceil_div(nch, S);
     p.S = (int)ceil_div(nch, p.cps);
-    p.UN = 8 / p.R;
-    p.smem = (size_t)p.cps * 64;
-    p.ws_bytes = p.S > 1 ? (int64_t)p.S * M * N * 4 : 0;
+    p.ws_bytes = p.S > 1 ? (int64_t)p.S * M * N * 4 + round_up(M * 4, 256) : 0;
     return p;
+}
+
+struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,ctas_per_sm,prefetch_tasks"
+    int G = 0, R = 0, ctas = 0, prefetch = -1;
+};
+
+const GemvTune &gemv_tune() {
+    static GemvTune t;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char *e = getenv("BITNET_GEMV_TUNE");
+        if (e != nullptr) sscanf(e, "%d,%d,%d,%d", &t.G, &t.R, &t.ctas, &t.prefetch);
+    });
+    return t;
 }
 
 using GemvKernel = void (*)(const GemvArgs);
 
-GemvKernel gemv_kernel_for(int G, int R, int *index) {
-    static const GemvKernel table[9] = {
-        gemv_w2a8_kernel<8, 4, 2>,  gemv_w2a8_kernel<8, 2, 4>,  gemv_w2a8_kernel<8, 1, 8>,
-        gemv_w2a8_kernel<16, 4, 2>, gemv_w2a8_kernel<16, 2, 4>, gemv_w2a8_kernel<16, 1, 8>,
-        gemv_w2a8_kernel<32, 4, 2>, gemv_w2a8_kernel<32, 2, 4>, gemv_w2a8_kernel<32, 1, 8>,
+GemvKernel gemv_kernel_for(int G, int R, int xmode, int *index) {
+    static const GemvKernel table[18] = {
+        gemv_w2a8_kernel<8, 1, 0>,  gemv_w2a8_kernel<8, 2, 0>,  gemv_w2a8_kernel<8, 4, 0>,
+        gemv_w2a8_kernel<16, 1, 0>, gemv_w2a8_kernel<16, 2, 0>, gemv_w2a8_kernel<16, 4, 0>,
+        gemv_w2a8_kernel<32, 1, 0>, gemv_w2a8_kernel<32, 2, 0>, gemv_w2a8_kernel<32, 4, 0>,
+        gemv_w2a8_kernel<8, 1, 1>,  gemv_w2a8_kernel<8, 2, 1>,  gemv_w2a8_kernel<8, 4, 1>,
+        gemv_w2a8_kernel<16, 1, 1>, gemv_w2a8_kernel<16, 2, 1>, gemv_w2a8_kernel<16, 4, 1>,
+        gemv_w2a8_kernel<32, 1, 1>, gemv_w2a8_kernel<32, 2, 1>, gemv_w2a8_kernel<32, 4, 1>,
     };
     const int gi = G == 8 ? 0 : (G == 16 ? 1 : 2);
-    const int ri = R == 4 ? 0 : (R == 2 ? 1 : 2);
-    *index = gi * 3 + ri;
+    const int ri = R == 1 ? 0 : (R == 2 ? 1 : 2);
+    *index = xmode * 9 + gi * 3 + ri;
     return table[*index];
 }
 
-int launch_gemv(DeviceInfo *dev, const int8_t *q, int64_t ldq, const uint8_t *packed, int64_t M, int64_t N,
-                int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
-                void *ws, cudaStream_t st) {
-    const GemvPlan p = plan_gemv(M, N, K);
+// Resident CTAs per SM of a GEMV instantiation at a given shared-memory size.
+int gemv_ctas_per_sm(DeviceInfo *dev, int idx, GemvKernel kern, size_t smem) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    for (int i = 0; i < dev->n_occ; ++i)
+        if (dev->occ[i].idx == idx && dev->occ[i].smem == smem) return dev->occ[i].ctas;
+    if (smem > 48 * 1024 && !(dev->smem_attr_set & (1u << idx))) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSliceChunks * 64) !=
+            cudaSuccess)
+            return -1;
+        dev->smem_attr_set |= 1u << idx;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess) return -1;
+    if (dev->n_occ < kOccCache) dev->occ[dev->n_occ++] = {idx, smem, n};
+    return n;
+}
+
+// xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
+// quantised per token inside the kernel.
+int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, int64_t ldq,
+                const uint8_t *packed, int64_t M, int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16,
+                const float *s_act, const float *gamma, void *ws, cudaStream_t st) {
+    const GemvSplit sp = plan_split(M, N, K);
+    const GemvTune &tn = gemv_tune();
+    int G = lanes_per_row(sp.cps);
+    if (tn.G == 8 || tn.G == 16 || tn.G == 32) G = tn.G;
+    const size_t smem = (size_t)sp.cps * 64;
+
+    // rows per lane group: the most that still give >= 2 tasks per resident warp
+    int idx = 0, R = 1;
+    for (int cand : {4, 2, 1}) {
+        GemvKernel k = gemv_kernel_for(G, cand, xmode, &idx);
+        const int c = gemv_ctas_per_sm(dev, idx, k, smem);
+        if (c <= 0) return BITNET_ERR_CUDA;
+        const int64_t warps = (int64_t)dev->sm_count * c * (kThreads / 32);
+        R = cand;
+        if (ceil_div(N, (32 / G) * cand) * M * sp.S >= 2 * warps) break;
+    }
+    if (tn.R == 1 || tn.R == 2 || tn.R == 4) R = tn.R;
+    GemvKernel kern = gemv_kernel_for(G, R, xmode, &idx);
+    int ctas = gemv_ctas_per_sm(dev, idx, kern, smem);
+    if (ctas <= 0) return BITNET_ERR_CUDA;
+    if (tn.ctas > 0 && tn.ctas < ctas) ctas = tn.ctas;
+
     GemvArgs a{};
-    a.q = q;
     a.ldq = ldq;
     a.W = packed;
     a.row_bytes = packed_row_bytes(K);
     a.N = N;
     a.K = K;
     a.nch_total = (int)(k_pad(K) / 64);
-    a.cps = p.cps;
-    a.M = (int)M;
-    a.y_i32 = y_i32;
-    a.y_bf16 = y_bf16;
-    a.partial = p.S > 1 ? static_cast<int32_t *>(ws) : nullptr;
-    a.s_act = s_act;
+    a.cps = sp.cps;
+    a.prefetch_tasks = tn.prefetch >= 0 ? tn.prefetch : 2;
     a.gamma = gamma;
+    int32_t *partial = sp.S > 1 ? static_cast<int32_t *>(ws) : nullptr;
+    float *s_out = (sp.S > 1 && xmode == 1)
+                       ? reinterpret_cast<float *>(static_cast<char *>(ws) + (int64_t)sp.S * M * N * 4)
+                       : nullptr;
 
-    int idx = 0;
-    GemvKernel kern = gemv_kernel_for(p.G, p.R, &idx);
-    if (p.smem > 48 * 1024) {
-        std::lock_guard<std::mutex> lk(g_dev_mu);
-        if (!(dev->smem_attr_set & (1u << idx))) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSliceChunks * 64) !=
-                cudaSuccess)
-                return BITNET_ERR_CUDA;
-            dev->smem_attr_set |= 1u << idx;
-        }
-    }
-    const int64_t row_tasks = ceil_div(N, (32 / p.G) * p.R);
+    const int64_t row_tasks = ceil_div(N, (32 / G) * R);
     // tokens go to gridDim.z (at most 65535 per launch)
     for (int64_t m0 = 0; m0 < M; m0 += 65535) {
         const int64_t mc = M - m0 < 65535 ? M - m0 : 65535;
         GemvArgs c = a;
-        c.q = q + m0 * ldq;
+        c.q = q ? q + m0 * ldq : nullptr;
+        c.x = x ? x + m0 * K : nullptr;
         c.M = (int)mc;
         c.y_i32 = y_i32 ? y_i32 + m0 * N : nullptr;
         c.y_bf16 = y_bf16 ? y_bf16 + m0 * N : nullptr;
         c.s_act = s_act ? s_act + m0 : nullptr;
+        c.partial = partial;
+        c.s_out = s_out ? s_out + m0 : nullptr;
         int64_t gx = ceil_div(row_tasks, kThreads / 32);
-        const int64_t cap = ceil_div((int64_t)dev->sm_count * 4, (int64_t)p.S * mc);
+        const int64_t cap = ceil_div((int64_t)dev->sm_count * ctas, (int64_t)sp.S * mc);
         if (gx > cap) gx = cap;
         if (gx < 1) gx = 1;
-        dim3 grid((unsigned)gx, (unsigned)p.S, (unsigned)mc);
-        kern<<<grid, kThreads, p.smem, st>>>(c);
-        int rc = launched();
+        const dim3 grid((unsigned)gx, (unsigned)sp.S, (unsigned)mc);
+        int rc = launched(launch_pdl(kern, grid, dim3(kThreads), smem, st, c));
         if (rc != BITNET_OK) return rc;
-        if (p.S > 1) {
-            gemv_splitk_reduce_kernel<<<grid_for(mc * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(c, p.S);
-            if ((rc = launched()) != BITNET_OK) return rc;
+        if (sp.S > 1) {
+            rc = launched(launch_pdl(gemv_splitk_reduce_kernel, dim3(grid_for(mc * N, kThreads * 4, dev->sm_count)),
+                                     dim3(kThreads), (size_t)0, st, c, sp.S));
+            if (rc != BITNET_OK) return rc;
         }
     }
     return BITNET_OK;
 }
-
-int64_t bitlinear_q_bytes(int64_t M, int64_t K) { return round_up(M * K, 256); }
 
 }  // namespace
 }  // namespace bitnet
@@ -205,11 +276,8 @@ BITNET_API int64_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (!sizes_ok(M, N, K)) return -1;
     int64_t need = (int64_t)kAbsmeanMaxBlocks * 8;  // bitnet_absmean partials
     if (M > 0 && N > 0 && K > 0) {
-        const int64_t g = plan_gemv(M, N, K).ws_bytes;
-        int64_t gemm = g;
-        int64_t bl = bitlinear_q_bytes(M, K) + round_up(M * 4, 256) + g;
-        if (gemm > need) need = gemm;
-        if (bl > need) need = bl;
+        const int64_t g = plan_split(M, N, K).ws_bytes;
+        if (g > need) need = g;
     }
     return need;
 }
@@ -284,7 +352,7 @@ BITNET_API int bitnet_w2a8_gemm(const int8_t *q, const uint8_t *packed, int32_t 
     if (M == 0 || N == 0) return BITNET_OK;
     if (y == nullptr || (K > 0 && (q == nullptr || packed == nullptr))) return BITNET_ERR_INVALID_ARG;
     if (!aligned(packed, 16) || !aligned(y, 4)) return BITNET_ERR_ALIGNMENT;
-    const int64_t need = K > 0 ? plan_gemv(M, N, K).ws_bytes : 0;
+    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BITNET_ERR_WORKSPACE;
     if (need > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
     DeviceInfo *dev = nullptr;
@@ -295,7 +363,7 @@ BITNET_API int bitnet_w2a8_gemm(const int8_t *q, const uint8_t *packed, int32_t 
         fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    return launch_gemv(dev, q, K, packed, M, N, K, y, nullptr, nullptr, nullptr, workspace, st);
+    return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, y, nullptr, nullptr, nullptr, workspace, st);
 }
 
 BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const float *gamma, uint16_t *y, int64_t M,
@@ -305,26 +373,19 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     if (y == nullptr || gamma == nullptr || (K > 0 && (x == nullptr || packed == nullptr)))
         return BITNET_ERR_INVALID_ARG;
     if (!aligned(x, 2) || !aligned(packed, 16) || !aligned(y, 2) || !aligned(gamma, 4)) return BITNET_ERR_ALIGNMENT;
+    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BITNET_ERR_WORKSPACE;
+    if (need > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
     DeviceInfo *dev = nullptr;
+    int rc = device_info(&dev);
+    if (rc != BITNET_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (K == 0) {
-        int rc = device_info(&dev);
-        if (rc != BITNET_OK) return rc;
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    const int64_t qb = bitlinear_q_bytes(M, K), sb = round_up(M * 4, 256);
-    const int64_t gw = plan_gemv(M, N, K).ws_bytes;
-    if (workspace == nullptr || workspace_bytes < qb + sb + gw) return BITNET_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
-    int rc = device_info(&dev);
-    if (rc != BITNET_OK) return rc;
-    int8_t *q = static_cast<int8_t *>(workspace);
-    float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + qb);
-    void *rest = static_cast<char *>(workspace) + qb + sb;
-    quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, K, false, s, nullptr);
-    if ((rc = launched()) != BITNET_OK) return rc;
-    return launch_gemv(dev, q, K, packed, M, N, K, nullptr, y, s, gamma, rest, st);
+    // activations are quantised per token inside the GEMV: one launch
+    return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
 }
 
 BITNET_API int bitnet_get_device_error(void *stream) {

@@ -41,6 +41,20 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
     return v;
 }
 
+// Asks the L2 to fetch [p, p + bytes) from HBM (16-byte aligned address and
+// size); nothing is returned to the thread and no completion is tracked.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before its predecessor on the stream finishes;
+// pdl_wait() blocks until that predecessor has completed and its writes are
+// visible.  pdl_launch_dependents() lets the successor start early.  Both are
+// no-ops for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
     return __uint_as_float(((uint32_t)h) << 16);
 }

@@ -89,13 +89,14 @@ def test_gemm_argument_errors(lib):
 
 
 def test_bitlinear_argument_errors(lib):
+    # every call here fails its host-side checks: none may reach a launch
     f = lib.bitnet_bitlinear
-    ws_need = lib.bitnet_workspace_bytes(2, 8, 64)
-    assert f(A, A, NULL, A, 2, 8, 64, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
-    assert f(MIS, A, A, A, 2, 8, 64, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
-    assert f(A, A, A, A, 2, 8, 64, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 2, 8, 64, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 2, 8, 64, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    ws_need = lib.bitnet_workspace_bytes(1, 64, 65536)  # a split-K shape: needs workspace
+    assert f(A, A, NULL, A, 1, 64, 65536, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
+    assert f(MIS, A, A, A, 1, 64, 65536, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    assert f(A, A, A, A, 1, 64, 65536, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 1, 64, 65536, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 1, 64, 65536, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
     assert f(NULL, NULL, NULL, NULL, 0, 8, 64, NULL, 0, S) == bn.BITNET_OK
 
 
