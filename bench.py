@@ -210,12 +210,9 @@ class GemvSet:
 
 
 def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
-    """Headline: one event-free graph per rotation copy (one step each, so
-    programmatic dependent launch links the calls), replayed round-robin.
-    Per-launch durations: a second timed loop over graphs with timing events
-    around every call (events between calls also break the launch overlap, so
-    these durations are conservative)."""
-    torch = gs.torch
+    """Headline: one graph per rotation copy holding one step (the calls of all
+    shapes back to back, linked by programmatic dependent launch), replayed
+    round-robin for exactly `steps` steps."""
     n_before = bn.bitnet_launch_count()
     graphs = [capture(torch, lambda c=c: gs.run(c)) for c in range(len(gs.copies))]
     launches_per_step = (bn.bitnet_launch_count() - n_before) // (2 * len(gs.copies))
@@ -224,25 +221,25 @@ def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
     ms = timed_graph_loop(torch, graphs, steps, warmup, dist)
     clk = clocks.stop() if clocks is not None else None
     del graphs
-    evs, egraphs = [], []
-    for c in range(len(gs.copies)):
-        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in gs.shapes]
-        egraphs.append(capture(torch, lambda c=c, ev=ev: gs.run(c, ev)))
-        evs.append(ev)
-    n_ev = max(len(gs.copies), min(steps, 20 * len(gs.copies)))
-    per_shape = [[] for _ in gs.shapes]
-    for i in range(n_ev):
-        c = i % len(gs.copies)
-        egraphs[c].replay()
-        if c == len(gs.copies) - 1:
-            torch.cuda.synchronize()
-            for cc in range(len(gs.copies)):
-                for j in range(len(gs.shapes)):
-                    per_shape[j].append(evs[cc][j][0].elapsed_time(evs[cc][j][1]) * 1e3)
-    torch.cuda.synchronize()
-    per_shape_us = [float(np.mean(d)) if d else float("nan") for d in per_shape]
-    del egraphs
-    return ms, per_shape_us, launches_per_step, clk
+    return ms, launches_per_step, clk
+
+
+def per_launch_us(torch, bn, gs, warmup, reps=30):
+    """Average duration of one call of each shape: a graph of back-to-back calls
+    of that shape over the rotating weight copies (each copy last read more than
+    2x L2 capacity earlier), timed with CUDA events on the capturing stream."""
+    out = []
+    C = len(gs.copies)
+    for j, (N, K) in enumerate(gs.shapes):
+        L = 4 * C
+        def run(j=j, N=N, L=L):
+            for i in range(L):
+                bn.bitnet_w2a8_gemm(gs.q[j], gs.copies[i % C][j], N, y=gs.y[j], ws=gs.ws[j])
+        g = capture(torch, run)
+        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+        out.append(ms * 1e3 / (reps * L))
+        del g
+    return out
 
 
 def e2e_sweep(torch, bn, gs, steps):
@@ -273,7 +270,10 @@ def e2e_sweep(torch, bn, gs, steps):
     return ms, h2d, d2h
 
 
-def measure_bitlinear_decode(torch, bn, shapes, steps, warmup, l2_bytes):
+def measure_bitlinear_decode(torch, bn, shapes, warmup, l2_bytes, reps=30):
+    """Fused BitLinear decode (bf16 in, bf16 out, weights ternarised and packed
+    on the GPU): mean per-call time in a graph of back-to-back calls over
+    rotating weight copies."""
     out = []
     for (N, K) in shapes:
         x, W = synth.bitlinear_inputs(1, N, K, seed=0)
@@ -281,17 +281,22 @@ def measure_bitlinear_decode(torch, bn, shapes, steps, warmup, l2_bytes):
         gamma = bn.bitnet_absmean(Wd)
         packed = bn.bitnet_pack_weights(bn.bitnet_ternarize(Wd, gamma))
         del Wd
-        c = rotation_copies(packed.numel(), l2_bytes)
-        copies = [packed] + [packed.clone() for _ in range(c - 1)]
+        C = rotation_copies(packed.numel(), l2_bytes)
+        copies = [packed] + [packed.clone() for _ in range(C - 1)]
         xd = bf16_dev(torch, x)
         y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
         ws = bn.workspace(1, N, K)
-        graphs = [capture(torch, lambda p=p: bn.bitnet_bitlinear(xd, p, gamma, N, y=y, ws=ws)) for p in copies]
-        ms = timed_graph_loop(torch, graphs, steps, warmup)
-        us = ms * 1e3 / steps
+        L = 4 * C
+
+        def run():
+            for i in range(L):
+                bn.bitnet_bitlinear(xd, copies[i % C], gamma, N, y=y, ws=ws)
+        g = capture(torch, run)
+        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+        us = ms * 1e3 / (reps * L)
         out.append({"N": N, "K": K, "us_per_call": round(us, 3),
                     "GBps": round(bitlinear_bytes(1, N, K) / (us * 1e-6) / 1e9, 1)})
-        del graphs, copies
+        del g, copies
     return out
 
 
@@ -338,8 +343,8 @@ def run_ours(args, rank, world, dist):
 
     gs = GemvSet(torch, bn, synth.SWEEP_SHAPES, synth.uniform_int8_ternary, seed=rank, l2_bytes=l2)
     clocks = ClockSampler(gpu_id_for(torch, dev)) if rank == 0 else None
-    ms, per_shape_us, launches_per_step, clk = measure_gemv_set(torch, bn, gs, args.steps, args.warmup, dist,
-                                                                clocks)
+    ms, launches_per_step, clk = measure_gemv_set(torch, bn, gs, args.steps, args.warmup, dist, clocks)
+    per_shape_us = per_launch_us(torch, bn, gs, args.warmup)
     ms_per_step = ms / args.steps
     value = world * gs.bytes_per_step * args.steps / (ms * 1e-3) / 1e9
     kern_us = sum(per_shape_us)
@@ -361,8 +366,7 @@ def run_ours(args, rank, world, dist):
     torch.cuda.empty_cache()
     if not args.quick and rank == 0:
         gl = GemvSet(torch, bn, synth.LARGE_SHAPES, synth.sparse_ternary_normal_int8, seed=0, l2_bytes=l2)
-        n = max(20, min(args.steps, 2000))
-        _, us_l, _, _ = measure_gemv_set(torch, bn, gl, n, max(3, args.warmup))
+        us_l = per_launch_us(torch, bn, gl, args.warmup)
         details["large"] = [{"N": N, "K": K, "us_per_call": round(u, 3),
                              "GBps": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9, 1),
                              "frac_hbm": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9 / hbm_peak, 4)}
@@ -370,7 +374,7 @@ def run_ours(args, rank, world, dist):
         del gl
         torch.cuda.empty_cache()
         details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
-                                                               max(20, min(args.steps, 2000)), max(3, args.warmup), l2)
+                                                               args.warmup, l2)
         details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES,
                                              max(10, min(args.steps // 20, 200)), max(3, args.warmup), int8_peak)
         details["int8_peak_tops"] = {"value": round(int8_peak, 1),
@@ -391,8 +395,10 @@ def run_ours(args, rank, world, dist):
                    "seed": "rank"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "kernel": "gemv_w2a8_kernel", "peak_source": peaks["source"],
-                     "per_launch_bytes": "N*K/4 + K + 4N per shape, mean over the 8 shapes"},
+                     "kernel": "gemv_tma_kernel", "peak_source": peaks["source"],
+                     "per_launch_bytes": "N*K/4 + K + 4N per shape, mean over the 8 shapes",
+                     "duration": "mean per-call time of each shape in a graph of back-to-back calls over rotating "
+                                 "weight copies (CUDA events)"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_tma.cuh"
 #include "quant.cuh"
 #include "weights.cuh"
 
@@ -32,7 +33,9 @@ struct DeviceInfo {
     bool init = false;
     int status = BITNET_OK;
     int sm_count = 0;
-    unsigned smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
+    uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
+    size_t tma_max_dyn[6] = {0, 0, 0, 0, 0, 0};  // dynamic shared memory opted into by each TMA GEMV
+    size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
     OccEntry occ[kOccCache];     // resident CTAs per SM by (instantiation, shared memory)
 };
@@ -50,8 +53,12 @@ int device_info(DeviceInfo **out) {
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BITNET_ERR_CUDA;
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return BITNET_ERR_CUDA;
         d.status = (major == 10) ? BITNET_OK : BITNET_ERR_UNSUPPORTED;
         d.sm_count = sms;
+        d.smem_optin = (size_t)optin;
         d.init = true;
     }
     *out = &d;
@@ -108,6 +115,20 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
+struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma"
+    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1;
+};
+
+const GemvTune &gemv_tune() {
+    static GemvTune t;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char *e = getenv("BITNET_GEMV_TUNE");
+        if (e != nullptr) sscanf(e, "%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma);
+    });
+    return t;
+}
+
 inline int lanes_per_row(int nch) { return nch >= 128 ? 32 : (nch >= 48 ? 16 : 8); }
 
 GemvSplit plan_split(int64_t M, int64_t N, int64_t K) {
@@ -120,53 +141,43 @@ GemvSplit plan_split(int64_t M, int64_t N, int64_t K) {
     // keeps >= 4 chunks per slice (small problems are latency-bound: a second
     // launch would cost more than it saves)
     while (tasks * S < kPlanSlots / 4 && nch / (2 * S) >= 4 * G) S *= 2;
+    if (gemv_tune().S > 0) S = gemv_tune().S;
     p.cps = (int)ceil_div(nch, S);
     p.S = (int)ceil_div(nch, p.cps);
     p.ws_bytes = p.S > 1 ? (int64_t)p.S * M * N * 4 + round_up(M * 4, 256) : 0;
     return p;
 }
 
-struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,ctas_per_sm,prefetch_tasks"
-    int G = 0, R = 0, ctas = 0, prefetch = -1;
-};
-
-const GemvTune &gemv_tune() {
-    static GemvTune t;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        const char *e = getenv("BITNET_GEMV_TUNE");
-        if (e != nullptr) sscanf(e, "%d,%d,%d,%d", &t.G, &t.R, &t.ctas, &t.prefetch);
-    });
-    return t;
-}
-
 using GemvKernel = void (*)(const GemvArgs);
 
-GemvKernel gemv_kernel_for(int G, int R, int xmode, int *index) {
-    static const GemvKernel table[18] = {
-        gemv_w2a8_kernel<8, 1, 0>,  gemv_w2a8_kernel<8, 2, 0>,  gemv_w2a8_kernel<8, 4, 0>,
-        gemv_w2a8_kernel<16, 1, 0>, gemv_w2a8_kernel<16, 2, 0>, gemv_w2a8_kernel<16, 4, 0>,
-        gemv_w2a8_kernel<32, 1, 0>, gemv_w2a8_kernel<32, 2, 0>, gemv_w2a8_kernel<32, 4, 0>,
-        gemv_w2a8_kernel<8, 1, 1>,  gemv_w2a8_kernel<8, 2, 1>,  gemv_w2a8_kernel<8, 4, 1>,
-        gemv_w2a8_kernel<16, 1, 1>, gemv_w2a8_kernel<16, 2, 1>, gemv_w2a8_kernel<16, 4, 1>,
-        gemv_w2a8_kernel<32, 1, 1>, gemv_w2a8_kernel<32, 2, 1>, gemv_w2a8_kernel<32, 4, 1>,
+// (R, U) pairs: rows per lane group x chunks per load batch
+constexpr int kRU[6][2] = {{1, 4}, {1, 8}, {2, 2}, {2, 4}, {4, 1}, {4, 2}};
+
+#define BITNET_GEMV_ROW(X, G)                                                                           \
+    gemv_w2a8_kernel<G, 1, 4, X>, gemv_w2a8_kernel<G, 1, 8, X>, gemv_w2a8_kernel<G, 2, 2, X>,          \
+        gemv_w2a8_kernel<G, 2, 4, X>, gemv_w2a8_kernel<G, 4, 1, X>, gemv_w2a8_kernel<G, 4, 2, X>
+
+GemvKernel gemv_kernel_for(int G, int ru, int xmode, int *index) {
+    static const GemvKernel table[36] = {
+        BITNET_GEMV_ROW(0, 8), BITNET_GEMV_ROW(0, 16), BITNET_GEMV_ROW(0, 32),
+        BITNET_GEMV_ROW(1, 8), BITNET_GEMV_ROW(1, 16), BITNET_GEMV_ROW(1, 32),
     };
     const int gi = G == 8 ? 0 : (G == 16 ? 1 : 2);
-    const int ri = R == 1 ? 0 : (R == 2 ? 1 : 2);
-    *index = xmode * 9 + gi * 3 + ri;
+    *index = xmode * 18 + gi * 6 + ru;
     return table[*index];
 }
+#undef BITNET_GEMV_ROW
 
 // Resident CTAs per SM of a GEMV instantiation at a given shared-memory size.
 int gemv_ctas_per_sm(DeviceInfo *dev, int idx, GemvKernel kern, size_t smem) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     for (int i = 0; i < dev->n_occ; ++i)
         if (dev->occ[i].idx == idx && dev->occ[i].smem == smem) return dev->occ[i].ctas;
-    if (smem > 48 * 1024 && !(dev->smem_attr_set & (1u << idx))) {
+    if (smem > 48 * 1024 && !(dev->smem_attr_set & (1ull << idx))) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSliceChunks * 64) !=
             cudaSuccess)
             return -1;
-        dev->smem_attr_set |= 1u << idx;
+        dev->smem_attr_set |= 1ull << idx;
     }
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess) return -1;
@@ -174,11 +185,111 @@ int gemv_ctas_per_sm(DeviceInfo *dev, int idx, GemvKernel kern, size_t smem) {
     return n;
 }
 
+// ------------------------------------------------------------------ TMA GEMV
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+
+// TMA GEMV variants: (warps per CTA, boxes in flight per warp)
+constexpr int kTmaCfg[3][2] = {{8, 4}, {12, 3}, {16, 2}};
+using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
+
+TmaKernel tma_kernel_for(int xmode, int cfg) {
+    static const TmaKernel table[6] = {gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 12, 3>, gemv_tma_kernel<0, 16, 2>,
+                                       gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 12, 3>, gemv_tma_kernel<1, 16, 2>};
+    return table[xmode * 3 + cfg];
+}
+
+// Opts a TMA GEMV variant into the largest dynamic shared memory left beside
+// its static shared memory; returns that size (0 on failure).
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    size_t &slot = dev->tma_max_dyn[xmode * 3 + cfg];
+    if (slot == 0) {
+        TmaKernel kern = tma_kernel_for(xmode, cfg);
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
+        const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess) return 0;
+        slot = dyn;
+    }
+    return slot;
+}
+
+// Shared memory the TMA GEMV needs for this shape on this device, or 0 if it
+// does not apply (then the register-streaming GEMV runs).
+size_t tma_plan(DeviceInfo *dev, int xmode, int64_t M, int64_t N, int64_t K, int *cfg, int *slices, int *max_blocks,
+                int *grid) {
+    const int tune = gemv_tune().tma;
+    if (M != 1 || tune == 0 || K < kTmaSliceK) return 0;
+    const int64_t row_bytes = packed_row_bytes(K);
+    const int64_t nblocks = ceil_div(N, kTmaRows);
+    const int64_t g = nblocks < dev->sm_count ? nblocks : dev->sm_count;
+    *slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
+    *max_blocks = (int)ceil_div(nblocks, g);
+    *grid = (int)g;
+    // measured on B200: more warps with fewer boxes each win once every SM
+    // has several row blocks; long rows prefer 12 x 3; small problems 8 x 4
+    if (tune >= 1 && tune <= 3)
+        *cfg = tune - 1;
+    else
+        *cfg = nblocks >= 4 * (int64_t)dev->sm_count ? 2 : (*slices >= 32 ? 1 : 0);
+    const size_t smem = gemv_tma_smem_bytes(kTmaCfg[*cfg][0], kTmaCfg[*cfg][1], *slices, *max_blocks);
+    if (tensor_map_encoder() == nullptr || smem > tma_max_dynamic_smem(dev, xmode, *cfg)) return 0;
+    return smem;
+}
+
+int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t N,
+                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, int cfg, int slices,
+                    int max_blocks, int grid, size_t smem, cudaStream_t st) {
+    const int64_t row_bytes = packed_row_bytes(K);
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)kTmaSliceBytes, (cuuint32_t)kTmaRows};
+    const cuuint32_t estride[2] = {1, 1};
+    if (tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
+                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return BITNET_ERR_CUDA;
+    TmaKernel kern = tma_kernel_for(xmode, cfg);
+    GemvTmaArgs a{};
+    a.q = q;
+    a.x = x;
+    a.N = N;
+    a.K = K;
+    a.slices = slices;
+    a.blk_begin = 0;
+    a.nblocks = ceil_div(N, kTmaRows);
+    a.max_blocks_cta = max_blocks;
+    a.y_i32 = y_i32;
+    a.y_bf16 = y_bf16;
+    a.gamma = gamma;
+    return launched(launch_pdl(kern, dim3(grid), dim3(kTmaCfg[cfg][0] * 32), smem, st, map, a));
+}
+
 // xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
 // quantised per token inside the kernel.
 int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, int64_t ldq,
                 const uint8_t *packed, int64_t M, int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16,
                 const float *s_act, const float *gamma, void *ws, cudaStream_t st) {
+    {
+        int cfg = 0, slices = 0, max_blocks = 0, grid = 0;
+        const size_t smem = tma_plan(dev, xmode, M, N, K, &cfg, &slices, &max_blocks, &grid);
+        if (smem > 0 && ldq == K)
+            return launch_gemv_tma(dev, xmode, q, x, packed, N, K, y_i32, y_bf16, gamma, cfg, slices, max_blocks,
+                                   grid, smem, st);
+    }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();
     int G = lanes_per_row(sp.cps);
@@ -186,17 +297,21 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     const size_t smem = (size_t)sp.cps * 64;
 
     // rows per lane group: the most that still give >= 2 tasks per resident warp
-    int idx = 0, R = 1;
-    for (int cand : {4, 2, 1}) {
+    int idx = 0, ru = 0;
+    for (int cand : {5, 3, 0}) {  // (4,2), (2,4), (1,4)
         GemvKernel k = gemv_kernel_for(G, cand, xmode, &idx);
         const int c = gemv_ctas_per_sm(dev, idx, k, smem);
         if (c <= 0) return BITNET_ERR_CUDA;
         const int64_t warps = (int64_t)dev->sm_count * c * (kThreads / 32);
-        R = cand;
-        if (ceil_div(N, (32 / G) * cand) * M * sp.S >= 2 * warps) break;
+        ru = cand;
+        if (ceil_div(N, (32 / G) * kRU[cand][0]) * M * sp.S >= 2 * warps) break;
     }
-    if (tn.R == 1 || tn.R == 2 || tn.R == 4) R = tn.R;
-    GemvKernel kern = gemv_kernel_for(G, R, xmode, &idx);
+    if (tn.R > 0 || tn.U > 0) {
+        for (int i = 0; i < 6; ++i)
+            if (kRU[i][0] == tn.R && kRU[i][1] == tn.U) ru = i;
+    }
+    const int R = kRU[ru][0];
+    GemvKernel kern = gemv_kernel_for(G, ru, xmode, &idx);
     int ctas = gemv_ctas_per_sm(dev, idx, kern, smem);
     if (ctas <= 0) return BITNET_ERR_CUDA;
     if (tn.ctas > 0 && tn.ctas < ctas) ctas = tn.ctas;
@@ -209,7 +324,7 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     a.K = K;
     a.nch_total = (int)(k_pad(K) / 64);
     a.cps = sp.cps;
-    a.prefetch_tasks = tn.prefetch >= 0 ? tn.prefetch : 2;
+    a.prefetch_tasks = tn.prefetch >= 0 ? tn.prefetch : 1;
     a.gamma = gamma;
     int32_t *partial = sp.S > 1 ? static_cast<int32_t *>(ws) : nullptr;
     float *s_out = (sp.S > 1 && xmode == 1)

@@ -22,7 +22,7 @@
 //     activations' sum over a lane's chunks is computed once.
 //   - Weights: each warp asks the L2 for the rows of its tasks a few tasks
 //     ahead with one bulk prefetch (no registers held), then reads them with
-//     16-byte loads one chunk ahead of use.
+//     16-byte loads in batches of U chunks x R rows, all in flight at once.
 //   - Decode without shifts: (word & (3 << 2j) per byte) is the code scaled by
 //     4^j; dp4a(unsigned code bytes, signed activations) accumulates each j in
 //     its own register, combined by exact arithmetic shifts.  Codes are w + 1,
@@ -31,8 +31,10 @@
 //   - Split-K (gridDim.y > 1) writes int32 partials; a second kernel adds them
 //     in slice order and applies the epilogue.
 //   - Programmatic dependent launch: weights never depend on an earlier kernel,
-//     so their prefetch is issued before griddepcontrol.wait; activations are
-//     read, and outputs written, after it.
+//     so their prefetch and the first batch of loads are issued before
+//     griddepcontrol.wait; activations are read, and outputs written, after it.
+//     (An earlier kernel on the stream that lets dependents launch early must
+//     therefore not write the packed weights; this library's kernels never do.)
 #pragma once
 
 #include "common.cuh"
@@ -93,34 +95,95 @@ __device__ __forceinline__ void stage_q_int8(uint4 *qs, const int8_t *qrow, int6
 
 // Fused per-token quantisation (same arithmetic as quant_act_kernel): absmax
 // over the whole row, then the slice's codes into qs.  Returns the scale.
+// Thread t owns the 16-value pieces t, t + blockDim, ...; up to kHeld of them
+// stay in registers between the absmax pass and the quantise pass.
+__device__ __forceinline__ void quant16(const uint4 &lo, const uint4 &hi, float sc, uint4 &out) {
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int8_t a = quant_one(__uint_as_float(w[2 * i] << 16), sc);
+        const int8_t b = quant_one(__uint_as_float(w[2 * i] & 0xffff0000u), sc);
+        const int8_t c = quant_one(__uint_as_float(w[2 * i + 1] << 16), sc);
+        const int8_t d = quant_one(__uint_as_float(w[2 * i + 1] & 0xffff0000u), sc);
+        o[i] = (uint32_t)(uint8_t)a | ((uint32_t)(uint8_t)b << 8) | ((uint32_t)(uint8_t)c << 16) |
+               ((uint32_t)(uint8_t)d << 24);
+    }
+    out = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ float amax16(const uint4 &lo, const uint4 &hi, float m) {
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        m = fmaxf(m, fabsf(__uint_as_float(w[i] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(w[i] & 0xffff0000u)));
+    }
+    return m;
+}
+
+// 16 bf16 values of piece p of a row (zeros beyond K), as two 16-byte words.
+__device__ __forceinline__ void load_x16(const uint16_t *xrow, int64_t K, int64_t p, bool vec, uint4 &lo, uint4 &hi) {
+    const int64_t k0 = p * 16;
+    if (vec && k0 + 16 <= K) {
+        lo = *reinterpret_cast<const uint4 *>(xrow + k0);
+        hi = *reinterpret_cast<const uint4 *>(xrow + k0 + 8);
+    } else {
+        uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        for (int t = 0; t < 16 && k0 + t < K; ++t) w[t >> 1] |= (uint32_t)xrow[k0 + t] << (16 * (t & 1));
+        lo = make_uint4(w[0], w[1], w[2], w[3]);
+        hi = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
 __device__ __forceinline__ float stage_q_bf16(uint4 *qs, float *red, const uint16_t *xrow, int64_t K, int c0,
                                               int nch) {
+    constexpr int kHeld = 4;
     const bool vec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
-    const int64_t K8 = vec ? (K / 8) * 8 : 0;
+    const int64_t npieces = ceil_div(K, 16);
+    uint4 held[kHeld][2];
     float amax = 0.0f;
-    for (int64_t k = (int64_t)threadIdx.x * 8; k < K8; k += (int64_t)blockDim.x * 8) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(xrow + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xffff0000u)));
+    for (int h = 0; h < kHeld; ++h) {
+        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
+        if (p < npieces) {
+            load_x16(xrow, K, p, vec, held[h][0], held[h][1]);
+            amax = amax16(held[h][0], held[h][1], amax);
         }
     }
-    for (int64_t k = K8 + threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(bf16_bits_to_float(xrow[k])));
+    for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < npieces; p += blockDim.x) {
+        uint4 lo, hi;
+        load_x16(xrow, K, p, vec, lo, hi);
+        amax = amax16(lo, hi, amax);
+    }
     amax = block_reduce(amax, [](float u, float v) { return fmaxf(u, v); }, red);
     const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
-    for (int p = threadIdx.x; p < 4 * nch; p += blockDim.x) {
-        const int64_t k0 = (int64_t)c0 * 64 + (int64_t)p * 16;
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 4
-        for (int t = 0; t < 16; ++t) {
-            if (k0 + t < K) {
-                const int8_t qi = quant_one(bf16_bits_to_float(xrow[k0 + t]), sc);
-                w[t >> 2] |= (uint32_t)(uint8_t)qi << (8 * (t & 3));
-            }
+    // pieces of this slice: global piece index 4*c0 + pl, pl < 4*nch
+    const int64_t pbeg = (int64_t)c0 * 4, pend = pbeg + 4 * nch;
+#pragma unroll
+    for (int h = 0; h < kHeld; ++h) {
+        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
+        if (p >= pbeg && p < pend) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (p < npieces) quant16(held[h][0], held[h][1], sc, v);
+            const int pl = (int)(p - pbeg);
+            qs[(pl & 3) * nch + (pl >> 2)] = v;
         }
-        qs[(p & 3) * nch + (p >> 2)] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    // pieces of the slice not held in registers (beyond kHeld per thread)
+    {
+        int64_t first = threadIdx.x + (int64_t)kHeld * blockDim.x;
+        if (first < pbeg) first += ceil_div(pbeg - first, (int64_t)blockDim.x) * blockDim.x;
+        for (int64_t p = first; p < pend; p += blockDim.x) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (p < npieces) {
+                uint4 lo, hi;
+                load_x16(xrow, K, p, vec, lo, hi);
+                quant16(lo, hi, sc, v);
+            }
+            const int pl = (int)(p - pbeg);
+            qs[(pl & 3) * nch + (pl >> 2)] = v;
+        }
     }
     return sc;
 }
@@ -132,8 +195,21 @@ __device__ __forceinline__ int group_sum(int v) {
     return v;
 }
 
-template <int G, int R, int XMODE>
-__global__ void __launch_bounds__(kThreads, 2) gemv_w2a8_kernel(const GemvArgs a) {
+// Loads batch `i0` (chunks l + G*(i0 + j), j < U) of R rows into registers;
+// chunks past the lane's count are not loaded.
+template <int G, int R, int U>
+__device__ __forceinline__ void load_batch(uint4 (&wb)[U][R], const uint8_t *const (&p)[R], int i0, int iters) {
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+        if (i0 + j < iters) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) wb[j][r] = ldg_stream_v4(p[r] + (int64_t)(i0 + j) * G * 16);
+        }
+    }
+}
+
+template <int G, int R, int U, int XMODE>
+__global__ void __launch_bounds__(kThreads, (R * U > 4 ? 2 : 3)) gemv_w2a8_kernel(const GemvArgs a) {
     static_assert(G == 8 || G == 16 || G == 32, "lanes per row");
     static_assert(R >= 1 && R <= G, "rows per lane group");
     extern __shared__ uint4 qs[];
@@ -152,6 +228,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_w2a8_kernel(const GemvArgs a
     const int64_t t0 = (int64_t)blockIdx.x * kWarps + warp;
     const uint8_t *wbase = a.W + (int64_t)c0 * 16;
     const bool full_rows = (nch == a.nch_total);  // a task's rows form one contiguous block
+    // this lane's chunks: l + G*i for i < iters
+    const int nfull = nch / G;
+    const int iters = nfull + (l < nch - nfull * G ? 1 : 0);
 
     auto prefetch_task = [&](int64_t t) {
         if (t >= n_tasks) return;
@@ -163,23 +242,34 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_w2a8_kernel(const GemvArgs a
             prefetch_l2_bulk(wbase + (r0 + lane) * row_bytes, (uint32_t)(nch * 16));
         }
     };
-    for (int d = 0; d < a.prefetch_tasks; ++d) prefetch_task(t0 + d * tw);
+    auto row_ptrs = [&](int64_t t, const uint8_t *(&p)[R]) {
+        const int64_t nb = t * RT + grp * R;
+#pragma unroll
+        for (int r = 0; r < R; ++r) p[r] = wbase + (nb + r < N ? nb + r : N - 1) * row_bytes + l * 16;
+    };
+
+    // Weights do not depend on the previous kernel: start streaming them
+    // (L2 prefetch of the first tasks, first batch into registers) before
+    // waiting for it.
+    uint4 wb[U][R];
+    const uint8_t *p[R];
+    for (int d = 0; d <= a.prefetch_tasks; ++d) prefetch_task(t0 + d * tw);
+    if (t0 < n_tasks) {
+        row_ptrs(t0, p);
+        load_batch<G, R, U>(wb, p, 0, iters);
+    }
     pdl_launch_dependents();
     pdl_wait();  // activations may come from the previous kernel on the stream
 
     float sc = 0.0f;
     if (XMODE == 0) {
         stage_q_int8(qs, a.q + (int64_t)m * a.ldq, a.K, c0, nch);
-        __syncthreads();
     } else {
         sc = stage_q_bf16(qs, red, a.x + (int64_t)m * a.K, a.K, c0, nch);
         if (a.s_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) a.s_out[m] = sc;
-        __syncthreads();
     }
+    __syncthreads();
 
-    // this lane's chunks: l + G*i for i < iters
-    const int nfull = nch / G;
-    const int iters = nfull + (l < nch - nfull * G ? 1 : 0);
     int qsum = 0;
     for (int i = 0; i < iters; ++i) {
         const int u = l + G * i;
@@ -191,46 +281,33 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_w2a8_kernel(const GemvArgs a
     qsum = group_sum<G>(qsum);
 
     float f = 0.0f;  // BitLinear rescale factor gamma / s_m
-    if (a.y_bf16 != nullptr && a.partial == nullptr)
-        f = __fdiv_rn(*a.gamma, XMODE == 0 ? a.s_act[m] : sc);
+    if (a.y_bf16 != nullptr && a.partial == nullptr) f = __fdiv_rn(*a.gamma, XMODE == 0 ? a.s_act[m] : sc);
 
     for (int64_t t = t0; t < n_tasks; t += tw) {
-        prefetch_task(t + a.prefetch_tasks * tw);
-        const int64_t nb = t * RT + grp * R;
-        const uint8_t *p[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) p[r] = wbase + (nb + r < N ? nb + r : N - 1) * row_bytes + l * 16;
-
+        prefetch_task(t + (a.prefetch_tasks + 1) * tw);
+        if (t != t0) row_ptrs(t, p);
         int acc[R][4];
 #pragma unroll
         for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0;
-        uint4 cur[R];
-        if (iters > 0) {
+        for (int i0 = 0; i0 < iters; i0 += U) {
+            if (t != t0 || i0 != 0) load_batch<G, R, U>(wb, p, i0, iters);
 #pragma unroll
-            for (int r = 0; r < R; ++r) cur[r] = ldg_stream_v4(p[r]);
-        }
-        for (int i = 0; i < iters; ++i) {
-            uint4 nxt[R];
-            const bool more = i + 1 < iters;
-            if (more) {
+            for (int j = 0; j < U; ++j) {
+                if (i0 + j < iters) {
+                    const int u = l + G * (i0 + j);
+                    const uint4 x0 = qs[u], x1 = qs[nch + u], x2 = qs[2 * nch + u], x3 = qs[3 * nch + u];
 #pragma unroll
-                for (int r = 0; r < R; ++r) nxt[r] = ldg_stream_v4(p[r] + (int64_t)(i + 1) * G * 16);
-            }
-            const int u = l + G * i;
-            const uint4 x0 = qs[u], x1 = qs[nch + u], x2 = qs[2 * nch + u], x3 = qs[3 * nch + u];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                mac_word(acc[r], cur[r].x, x0);
-                mac_word(acc[r], cur[r].y, x1);
-                mac_word(acc[r], cur[r].z, x2);
-                mac_word(acc[r], cur[r].w, x3);
-            }
-            if (more) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) cur[r] = nxt[r];
+                    for (int r = 0; r < R; ++r) {
+                        mac_word(acc[r], wb[j][r].x, x0);
+                        mac_word(acc[r], wb[j][r].y, x1);
+                        mac_word(acc[r], wb[j][r].z, x2);
+                        mac_word(acc[r], wb[j][r].w, x3);
+                    }
+                }
             }
         }
 
+        const int64_t nb = t * RT + grp * R;
         int tot[R];
 #pragma unroll
         for (int r = 0; r < R; ++r)

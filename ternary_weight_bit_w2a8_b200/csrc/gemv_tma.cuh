@@ -1,0 +1,300 @@
+// gemv_tma.cuh -- the decode GEMV for large weight matrices: packed weights
+// stream through shared memory by TMA, one row per lane.
+//
+// Same contraction and decode as gemv.cuh (layout v1 words, shift-free dp4a
+// on codes scaled by 4^j, activation-sum correction); what differs is how the
+// weights reach the lanes:
+//   - The packed matrix is a 2-D byte tensor [N rows, K_pad/4 bytes].  A TMA
+//     box is 32 rows x 128 bytes (512 k) = 4 KB, written to shared memory with
+//     the 128-byte swizzle, so lane r reading 16-byte chunk c of its own row r
+//     (address r*128 + ((c ^ (r & 7)) * 16)) is free of bank conflicts.
+//   - Work items are (32-row block, 128-byte K-slice) pairs.  CTA b owns row
+//     blocks b, b + gridDim.x, ...; its items, in (row block, slice) order, are
+//     split into equal contiguous ranges, one per warp, which keeps every warp
+//     busy for any K and makes a warp leave a row block at most a few times.
+//   - Each warp has a private ring of NS boxes and one mbarrier per stage; its
+//     lane 0 issues the TMA for the item NS ahead as soon as the warp has read
+//     a stage, so up to NS boxes per warp are in flight without holding
+//     registers.
+//   - Activations live in shared memory as one linear array; all lanes read
+//     the same 16 bytes at a time (a broadcast).
+//   - A warp adds its per-row partial sums into a per-row-block int32
+//     accumulator in shared memory (atomics: exact and order-free) whenever its
+//     item sequence leaves a row block; the warp whose contribution completes
+//     the block's item count writes the 32 results.
+//   - Every mbarrier wait is bounded in time.  A warp that gives up records
+//     BITNET_ERR_DEVICE_TIMEOUT, waits (bounded) for its own boxes in flight and
+//     returns; that row block's outputs are then left unwritten.
+//   - Programmatic dependent launch as in gemv.cuh: the first boxes of every
+//     warp are requested before griddepcontrol.wait.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace bitnet {
+
+constexpr int kTmaRows = 32;                                // rows per box (one per lane)
+constexpr int kTmaSliceBytes = 128;                         // packed bytes per row per box
+constexpr int kTmaSliceK = kTmaSliceBytes * 4;              // k values per box
+constexpr int kTmaBoxBytes = kTmaRows * kTmaSliceBytes;     // 4 KB
+constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s per wait
+
+struct GemvTmaArgs {
+    const int8_t *q;      // int8 activations [M, K] (mode 0)
+    const uint16_t *x;    // bf16 activations [M, K] (mode 1)
+    int64_t N, K;
+    int slices;           // K-slices of 128 packed bytes per row
+    int64_t blk_begin;    // first row block of this launch
+    int64_t nblocks;      // row blocks of this launch
+    int max_blocks_cta;   // accumulator slots per CTA
+    int32_t *y_i32;       // [M, N] int32 result
+    uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
+    const float *gamma;   // weight scale (BitLinear)
+};
+
+// Dynamic shared memory of a launch: ring of warps x stages boxes, linear
+// activations, per-row-block accumulators and counters, mbarriers.
+__host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta) {
+    return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes + (size_t)slices * kTmaSliceK +
+           (size_t)max_blocks_cta * kTmaRows * 4 + (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for the phase of the given parity to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+__device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Linear staging of int8 activations: qlin[k] = q[k] for k < K, 0 up to kq.
+__device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, const int8_t *qrow, int64_t K, int64_t kq) {
+    const bool vec = ((reinterpret_cast<uintptr_t>(qrow) & 15) == 0);
+    for (int64_t k0 = (int64_t)threadIdx.x * 16; k0 < kq; k0 += (int64_t)blockDim.x * 16) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (vec && k0 + 16 <= K) {
+            v = *reinterpret_cast<const uint4 *>(qrow + k0);
+        } else if (k0 < K) {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            for (int t = 0; t < 16 && k0 + t < K; ++t) w[t >> 2] |= (uint32_t)(uint8_t)qrow[k0 + t] << (8 * (t & 3));
+            v = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *reinterpret_cast<uint4 *>(qlin + k0) = v;
+    }
+}
+
+// Linear staging with fused per-token quantisation of bf16 activations (same
+// arithmetic as quant_act_kernel).  Returns the scale.
+__device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, float *red, const uint16_t *xrow, int64_t K,
+                                                 int64_t kq) {
+    constexpr int kHeld = 4;
+    const bool vec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
+    const int64_t npieces = ceil_div(K, 16), qpieces = kq / 16;
+    uint4 held[kHeld][2];
+    float amax = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kHeld; ++h) {
+        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
+        if (p < npieces) {
+            load_x16(xrow, K, p, vec, held[h][0], held[h][1]);
+            amax = amax16(held[h][0], held[h][1], amax);
+        }
+    }
+    for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < npieces; p += blockDim.x) {
+        uint4 lo, hi;
+        load_x16(xrow, K, p, vec, lo, hi);
+        amax = amax16(lo, hi, amax);
+    }
+    amax = block_reduce(amax, [](float u, float v) { return fmaxf(u, v); }, red);
+    const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
+#pragma unroll
+    for (int h = 0; h < kHeld; ++h) {
+        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
+        if (p < qpieces) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (p < npieces) quant16(held[h][0], held[h][1], sc, v);
+            *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
+        }
+    }
+    for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < qpieces; p += blockDim.x) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (p < npieces) {
+            uint4 lo, hi;
+            load_x16(xrow, K, p, vec, lo, hi);
+            quant16(lo, hi, sc, v);
+        }
+        *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
+    }
+    return sc;
+}
+
+template <int XMODE, int W, int NS>
+__global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ float red[32];
+    // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8 rows
+    // of 128 bytes); computed on the shared-window address so that every
+    // pointer below stays a shared-memory pointer
+    uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * NS * kTmaBoxBytes);
+    const int64_t kq = (int64_t)a.slices * kTmaSliceK;
+    int *accs = reinterpret_cast<int *>(qlin + kq);
+    int *done = accs + a.max_blocks_cta * kTmaRows;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(done + a.max_blocks_cta + ((a.max_blocks_cta & 1) ? 1 : 0));
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slices = a.slices;
+    const int64_t nb_cta = a.nblocks > blockIdx.x ? ceil_div(a.nblocks - blockIdx.x, gridDim.x) : 0;
+    const int64_t items = nb_cta * slices;
+    // this warp's items: a contiguous range of (row block, slice) pairs
+    const int64_t ipw = ceil_div(items, W);
+    const int64_t it_begin = min(items, warp * ipw);
+    const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
+    uint64_t *mybar = bars + warp * NS;
+    uint8_t *myring = ring + warp * NS * kTmaBoxBytes;
+
+    if (threadIdx.x < W * NS) mbar_init(&bars[threadIdx.x], 1);
+    for (int64_t i = threadIdx.x; i < nb_cta * kTmaRows; i += blockDim.x) accs[i] = 0;
+    for (int64_t i = threadIdx.x; i < nb_cta; i += blockDim.x) done[i] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+
+    // issue cursor (lane 0 only): next item to request
+    int64_t ibl = it_begin / slices;
+    int ij = (int)(it_begin - ibl * slices);
+    auto issue_next = [&](int s) {
+        const int64_t row0 = (a.blk_begin + blockIdx.x + ibl * gridDim.x) * kTmaRows;
+        mbar_arrive_expect_tx(&mybar[s], kTmaBoxBytes);
+        tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
+        if (++ij == slices) {
+            ij = 0;
+            ++ibl;
+        }
+    };
+    // weights do not depend on the previous kernel: request them before waiting for it
+    if (lane == 0)
+        for (int s = 0; s < NS && s < n_items; ++s) issue_next(s);
+    pdl_launch_dependents();
+    pdl_wait();
+
+    float sc = 0.0f;
+    if (XMODE == 0)
+        stage_qlin_int8(qlin, a.q, a.K, kq);
+    else
+        sc = stage_qlin_bf16(qlin, red, a.x, a.K, kq);
+    __syncthreads();
+
+    int qsum = 0;
+    for (int64_t p = lane; p < kq / 16; p += 32) qsum = byte_sum(reinterpret_cast<const uint4 *>(qlin)[p], qsum);
+    qsum = group_sum<32>(qsum);
+    float f = 0.0f;
+    if (XMODE == 1) f = __fdiv_rn(*a.gamma, sc);
+
+    int acc[4] = {0, 0, 0, 0};
+    int ncontrib = 0;
+    // folds this warp's partial sums of row block `bl` into shared memory; the
+    // warp completing the block writes its 32 outputs
+    auto flush = [&](int64_t bl) {
+        const int v = acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6);
+        atomicAdd(&accs[bl * kTmaRows + lane], v);
+        __threadfence_block();
+        __syncwarp();
+        int fin = 0;
+        if (lane == 0) fin = (atomicAdd(&done[bl], ncontrib) + ncontrib == slices);
+        fin = __shfl_sync(0xffffffffu, fin, 0);
+        if (fin) {
+            __threadfence_block();
+            const int tot = atomicAdd(&accs[bl * kTmaRows + lane], 0);
+            const int64_t n = (a.blk_begin + blockIdx.x + bl * gridDim.x) * kTmaRows + lane;
+            if (n < a.N) {
+                const int r = tot - qsum;
+                if (XMODE == 1)
+                    a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)r, f));
+                else
+                    a.y_i32[n] = r;
+            }
+        }
+        acc[0] = acc[1] = acc[2] = acc[3] = 0;
+        ncontrib = 0;
+    };
+
+    // consume cursor
+    int64_t cbl = it_begin / slices;
+    int cj = (int)(it_begin - cbl * slices);
+    for (int n = 0; n < n_items; ++n) {
+        const int s = n % NS;
+        if (!mbar_wait_bounded(&mybar[s], (uint32_t)(n / NS) & 1u)) {
+            if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
+            // wait (bounded) for this warp's boxes still in flight, then leave
+            for (int d = 0; d < NS && n + d < n_items; ++d)
+                mbar_wait_bounded(&mybar[(n + d) % NS], (uint32_t)((n + d) / NS) & 1u);
+            return;
+        }
+        const uint8_t *row = myring + s * kTmaBoxBytes + lane * kTmaSliceBytes;
+        const int8_t *qk = qlin + cj * kTmaSliceK;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (lane & 7)) << 4));
+            const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
+            const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];
+            mac_word(acc, w.x, x0);
+            mac_word(acc, w.y, x1);
+            mac_word(acc, w.z, x2);
+            mac_word(acc, w.w, x3);
+        }
+        ++ncontrib;
+        __syncwarp();
+        if (lane == 0 && n + NS < n_items) issue_next(s);
+        if (++cj == slices || n + 1 == n_items) {
+            flush(cbl);
+            cj = 0;
+            ++cbl;
+        }
+    }
+}
+
+}  // namespace bitnet
