@@ -168,6 +168,34 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
                                 int64_t workspace_bytes, void *stream);
 
 /*
+ * Allocation-free variant of bitnet_w2a8_gemm.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory --
+ * for instance a host program that only receives device buffers from another
+ * framework and has no device allocator of its own, or a service whose device
+ * memory is fixed up front -- and so cannot provide the workspace that
+ * bitnet_w2a8_gemm may need.  Instead it uses one scratch array of
+ * BITNET_NOALLOC_SCRATCH_BYTES compiled into this library as a file-scope
+ * __device__ array, which every GPU that loads the library holds until the
+ * process exits.
+ *   Same arguments, layouts, result and errors as bitnet_w2a8_gemm, without
+ *   the workspace.  Returns BITNET_ERR_WORKSPACE (before any device work) when
+ *   the problem needs more scratch than BITNET_NOALLOC_SCRATCH_BYTES; many
+ *   shapes need none (bitnet_workspace_bytes(M, N, K) <= 8192 means the
+ *   contraction itself needs none).
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   All calls share the one array and it keeps the contents of the last call;
+ *   every call writes the scratch it reads, so nothing has to be cleared, but
+ *   calls that overlap on the GPU (other streams, other threads) race on it
+ *   and must be serialised by the caller.
+ *   No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define BITNET_NOALLOC_SCRATCH_BYTES 1048576
+BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M,
+                                        int64_t N, int64_t K, void *stream);
+
+/*
  * Device-side error word.  Kernels whose threads wait on one another bound
  * every wait; a wait that runs out records BITNET_ERR_DEVICE_TIMEOUT in a
  * per-device word (the kernel then stops and leaves its output incomplete).

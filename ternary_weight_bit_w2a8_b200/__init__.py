@@ -38,6 +38,7 @@ _SIGNATURES = {
     "bitnet_quant_act": (ctypes.c_int, [_p, _i64, _i64, _p, _p, _p, _p]),
     "bitnet_w2a8_gemm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, _i64, _p, _i64, _p]),
     "bitnet_bitlinear": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _i64, _p]),
+    "bitnet_w2a8_gemm_noalloc": (ctypes.c_int, [_p, _p, _p, _i64, _i64, _i64, _p]),
     "bitnet_get_device_error": (ctypes.c_int, [_p]),
     "bitnet_launch_count": (_i64, []),
 }
@@ -199,6 +200,20 @@ def bitnet_bitlinear(x, packed, gamma, N: int, y=None, ws=None, stream=None):
         ws = workspace(M, N, K, x.device)
     _check(lib().bitnet_bitlinear(_ptr(x), _ptr(packed), _ptr(gamma), _ptr(y), M, N, K, _ptr(ws), ws.numel(),
                                   _stream(stream)), "bitnet_bitlinear")
+    return y
+
+
+def bitnet_w2a8_gemm_noalloc(q, packed, N: int, y=None, stream=None):
+    """bitnet_w2a8_gemm without a workspace: for callers that cannot allocate
+    device memory.  Uses the library's one built-in scratch array (see the C
+    header): calls that overlap on the GPU race on it."""
+    import torch
+    _dev(q, "q")
+    M, K = q.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.int32, device=q.device)
+    _check(lib().bitnet_w2a8_gemm_noalloc(_ptr(q), _ptr(packed), _ptr(y), M, N, K, _stream(stream)),
+           "bitnet_w2a8_gemm_noalloc")
     return y
 
 

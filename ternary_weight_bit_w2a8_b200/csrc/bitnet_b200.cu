@@ -360,6 +360,27 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     return BITNET_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free scratch
+// Scratch of bitnet_w2a8_gemm_noalloc: one array per device, shared by every
+// call; its device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BITNET_NOALLOC_SCRATCH_BYTES];
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BITNET_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return BITNET_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return BITNET_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return BITNET_OK;
+}
+
 }  // namespace
 }  // namespace bitnet
 
@@ -501,6 +522,27 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     }
     // activations are quantised per token inside the GEMV: one launch
     return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
+}
+
+BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M, int64_t N,
+                                        int64_t K, void *stream) {
+    if (!sizes_ok(M, N, K)) return BITNET_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return BITNET_OK;
+    if (y == nullptr || (K > 0 && (q == nullptr || packed == nullptr))) return BITNET_ERR_INVALID_ARG;
+    if (!aligned(packed, 16) || !aligned(y, 4)) return BITNET_ERR_ALIGNMENT;
+    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
+    if (need > (int64_t)BITNET_NOALLOC_SCRATCH_BYTES) return BITNET_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    int rc = device_info(&dev);
+    if (rc != BITNET_OK) return rc;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != BITNET_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
+        return launched();
+    }
+    return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, y, nullptr, nullptr, nullptr, scratch, st);
 }
 
 BITNET_API int bitnet_get_device_error(void *stream) {

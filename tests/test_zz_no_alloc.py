@@ -1,0 +1,54 @@
+"""The allocation-free W2A8 GEMM entry point (bitnet_w2a8_gemm_noalloc).
+
+It serves callers that cannot allocate device memory and therefore cannot pass
+the workspace bitnet_w2a8_gemm may need; it uses the library's one built-in
+scratch array instead.  These tests call it through the C ABI and check it
+against the workspace entry point on the same inputs, two calls in a row with
+different data (the shared scratch keeps the previous call's contents, so a
+stale read would show), including a shape whose plan does use scratch.  This
+file is collected last on purpose.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import ternary_weight_bit_w2a8_b200 as bn
+from ternary_weight_bit_w2a8_b200 import synth
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    # checked on the host before any device work: fake pointers are never used
+    lib = bn.lib()
+    A = ctypes.c_void_p(0x10000)
+    M, N, K = 4, 65536, 131072
+    assert lib.bitnet_workspace_bytes(M, N, K) > 1048576
+    assert lib.bitnet_w2a8_gemm_noalloc(A, A, A, M, N, K, None) == bn.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_w2a8_gemm_noalloc(A, A, A, 0, N, K, None) == bn.BITNET_OK
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_two_calls():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = bn.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    # (2, 640, 131072) and (2, 64, 65536) split K and keep int32 partials in the
+    # scratch array; for the first, the partials alone exceed the 8 KiB that
+    # bitnet_workspace_bytes reserves for other entry points
+    cases = [(2, 640, 131072), (2, 64, 65536), (1, 300, 2560), (3, 129, 1000), (1, 7, 100)]
+    assert lib.bitnet_workspace_bytes(2, 640, 131072) > 8192
+    for (M, N, K) in cases:
+        for call in range(2):
+            q, w = synth.uniform_int8_ternary(N, K, seed=1000 * call + M + N, M=M)
+            qd = torch.from_numpy(q).cuda()
+            packed = bn.bitnet_pack_weights(torch.from_numpy(w).cuda())
+            y_ref = bn.bitnet_w2a8_gemm(qd, packed, N)
+            y = torch.full((M, N), -7, dtype=torch.int32, device="cuda")
+            rc = lib.bitnet_w2a8_gemm_noalloc(ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(packed.data_ptr()),
+                                              ctypes.c_void_p(y.data_ptr()), M, N, K, stream)
+            assert rc == bn.BITNET_OK, bn.status_string(rc)
+            torch.cuda.synchronize()
+            assert torch.equal(y, y_ref), (M, N, K, call)
+    assert bn.bitnet_get_device_error() == 0
