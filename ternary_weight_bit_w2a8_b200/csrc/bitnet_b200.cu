@@ -217,6 +217,16 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
     size_t &slot = dev->tma_max_dyn[xmode * 3 + cfg];
     if (slot == 0) {
         TmaKernel kern = tma_kernel_for(xmode, cfg);
+    // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
+    // makes one wait run out, exercising the device-timeout path
+    static std::atomic<int> stall_once{-1};
+    if (stall_once.load() == -1) {
+        const char *e = getenv("BITNET_TEST_STALL");
+        int expect = -1;
+        stall_once.compare_exchange_strong(expect, (e != nullptr && e[0] == '1') ? 1 : 0);
+    }
+    int one = 1;
+    const int test_stall = stall_once.compare_exchange_strong(one, 0) ? 1 : 0;
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -263,6 +273,16 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return BITNET_ERR_CUDA;
     TmaKernel kern = tma_kernel_for(xmode, cfg);
+    // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
+    // makes one wait run out, exercising the device-timeout path
+    static std::atomic<int> stall_once{-1};
+    if (stall_once.load() == -1) {
+        const char *e = getenv("BITNET_TEST_STALL");
+        int expect = -1;
+        stall_once.compare_exchange_strong(expect, (e != nullptr && e[0] == '1') ? 1 : 0);
+    }
+    int one = 1;
+    const int test_stall = stall_once.compare_exchange_strong(one, 0) ? 1 : 0;
     GemvTmaArgs a{};
     a.q = q;
     a.x = x;
@@ -275,6 +295,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
+    a.test_stall = test_stall;
     return launched(launch_pdl(kern, dim3(grid), dim3(kTmaCfg[cfg][0] * 32), smem, st, map, a));
 }
 

@@ -54,6 +54,7 @@ struct GemvTmaArgs {
     int32_t *y_i32;       // [M, N] int32 result
     uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
     const float *gamma;   // weight scale (BitLinear)
+    int test_stall;       // test hook: warp 0 never requests its first box, so its first wait times out
 };
 
 // Dynamic shared memory of a launch: ring of warps x stages boxes, linear
@@ -216,8 +217,18 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
         }
     };
     // weights do not depend on the previous kernel: request them before waiting for it
-    if (lane == 0)
-        for (int s = 0; s < NS && s < n_items; ++s) issue_next(s);
+    if (lane == 0) {
+        for (int s = 0; s < NS && s < n_items; ++s) {
+            if (s == 0 && warp == 0 && a.test_stall) {  // skip the request: nothing completes this stage
+                if (++ij == slices) {
+                    ij = 0;
+                    ++ibl;
+                }
+                continue;
+            }
+            issue_next(s);
+        }
+    }
     pdl_launch_dependents();
     pdl_wait();
 
@@ -269,8 +280,8 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
         const int s = n % NS;
         if (!mbar_wait_bounded(&mybar[s], (uint32_t)(n / NS) & 1u)) {
             if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
-            // wait (bounded) for this warp's boxes still in flight, then leave
-            for (int d = 0; d < NS && n + d < n_items; ++d)
+            // wait (bounded) for this warp's other boxes still in flight, then leave
+            for (int d = 1; d < NS && n + d < n_items; ++d)
                 mbar_wait_bounded(&mybar[(n + d) % NS], (uint32_t)((n + d) / NS) & 1u);
             return;
         }
