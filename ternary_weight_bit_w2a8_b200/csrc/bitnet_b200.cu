@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_tma.cuh"
+#include "gemm_tc.cuh"
 #include "quant.cuh"
 #include "weights.cuh"
 
@@ -35,6 +36,7 @@ struct DeviceInfo {
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
     size_t tma_max_dyn[6] = {0, 0, 0, 0, 0, 0};  // dynamic shared memory opted into by each TMA GEMV
+    bool tc_attr_set[8] = {false, false, false, false, false, false, false, false};
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
     OccEntry occ[kOccCache];     // resident CTAs per SM by (instantiation, shared memory)
@@ -402,6 +404,141 @@ int noalloc_scratch(void **out) {
     return BITNET_OK;
 }
 
+// ------------------------------------------------------------------ tcgen05 GEMM (M > 1)
+constexpr int kTcBNs[4] = {256, 128, 96, 64};
+using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmTcArgs);
+
+TcKernel tc_kernel_for(int bn_idx, bool bf16, size_t *smem) {
+    static const TcKernel k[8] = {gemm_w2a8_tc_kernel<256, false>, gemm_w2a8_tc_kernel<128, false>,
+                                  gemm_w2a8_tc_kernel<96, false>,  gemm_w2a8_tc_kernel<64, false>,
+                                  gemm_w2a8_tc_kernel<256, true>,  gemm_w2a8_tc_kernel<128, true>,
+                                  gemm_w2a8_tc_kernel<96, true>,   gemm_w2a8_tc_kernel<64, true>};
+    static const size_t sz[4] = {TcSmem<256>::kBytes + 1024, TcSmem<128>::kBytes + 1024,
+                                 TcSmem<96>::kBytes + 1024, TcSmem<64>::kBytes + 1024};
+    *smem = sz[bn_idx];
+    return k[(bf16 ? 4 : 0) + bn_idx];
+}
+
+// Weight rows per tile: the largest tile that still gives every SM a tile.
+int tc_bn_index(int64_t M, int64_t N, int sm_count) {
+    const int64_t mt = ceil_div(M, kTcBM);
+    for (int i = 0; i < 4; ++i)
+        if (mt * ceil_div(N, kTcBNs[i]) >= sm_count) return i;
+    return 3;
+}
+
+int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t *packed, int64_t M, int64_t N,
+                   int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
+                   cudaStream_t st) {
+    const GemvTune &tn = gemv_tune();
+    int bi = tc_bn_index(M, N, dev->sm_count);
+    if (tn.R < 0 && -tn.R <= 4) bi = -tn.R - 1;  // tuning override: R = -1..-4 picks the tile width
+    const int BN = kTcBNs[bi];
+    const bool bf16 = y_bf16 != nullptr;
+    size_t smem = 0;
+    TcKernel kern = tc_kernel_for(bi, bf16, &smem);
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        bool &set = dev->tc_attr_set[(bf16 ? 4 : 0) + bi];
+        if (!set) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return BITNET_ERR_CUDA;
+            set = true;
+        }
+    }
+    CUtensorMap amap, pmap;
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)lda};
+        const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBM};
+        const cuuint32_t es[2] = {1, 1};
+        if (tensor_map_encoder()(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(q), gdim, gstride, box,
+                                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BITNET_ERR_CUDA;
+    }
+    {
+        const int64_t row_bytes = packed_row_bytes(K);
+        const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
+        const cuuint32_t box[2] = {32u, (cuuint32_t)BN};
+        const cuuint32_t es[2] = {1, 1};
+        if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
+                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BITNET_ERR_CUDA;
+    }
+    GemmTcArgs a{};
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.nk = (int)(k_pad(K) / kTcBK);
+    a.y_i32 = y_i32;
+    a.y_bf16 = y_bf16;
+    a.s_act = s_act;
+    a.gamma = gamma;
+    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)ceil_div(M, kTcBM));
+    return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, a));
+}
+
+// Copies int8 activations [M, K] into rows of K_pad bytes, zero-padded, so the
+// tensor map's row stride is a multiple of 16 bytes.
+__global__ void __launch_bounds__(kThreads) repack_q_kernel(const int8_t *__restrict__ q, int64_t M, int64_t K,
+                                                            int64_t ld, int8_t *__restrict__ out) {
+    const int64_t total = M * ld;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += (int64_t)gridDim.x * kThreads) {
+        const int64_t m = i / ld, k = i - m * ld;
+        out[i] = k < K ? q[m * K + k] : (int8_t)0;
+    }
+}
+
+// ------------------------------------------------------------------ dispatch
+// One plan for every caller of the contraction, so the path taken and the
+// scratch it needs always agree.
+enum { kPathGemv = 0, kPathTc = 1 };
+struct GemmPlan {
+    int path;
+    bool repack;       // int8 activations copied to K_pad-strided rows first
+    int64_t ws_bytes;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinear) {
+    GemmPlan p{};
+    if (M >= 2 && K >= kTcBK && tensor_map_encoder() != nullptr) {
+        p.path = kPathTc;
+        const int64_t qbytes = round_up(M * k_pad(K), 256);
+        if (bitlinear) {
+            p.ws_bytes = qbytes + round_up(M * 4, 256);
+        } else {
+            p.repack = !q_tma_ok;
+            p.ws_bytes = p.repack ? qbytes : 0;
+        }
+    } else {
+        p.path = kPathGemv;
+        p.ws_bytes = plan_split(M, N, K).ws_bytes;
+    }
+    return p;
+}
+
+// The whole int32 contraction for M, N, K >= 1 (validated by the caller).
+int run_w2a8_gemm(DeviceInfo *dev, const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M, int64_t N,
+                  int64_t K, void *ws, const GemmPlan &p, cudaStream_t st) {
+    if (p.path == kPathGemv) return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, y, nullptr, nullptr, nullptr, ws, st);
+    const int8_t *qa = q;
+    int64_t lda = K;
+    if (p.repack) {
+        int8_t *qp = static_cast<int8_t *>(ws);
+        lda = k_pad(K);
+        repack_q_kernel<<<grid_for(M * lda, kThreads * 8, dev->sm_count), kThreads, 0, st>>>(q, M, K, lda, qp);
+        const int rc = launched();
+        if (rc != BITNET_OK) return rc;
+        qa = qp;
+    }
+    return launch_gemm_tc(dev, qa, lda, packed, M, N, K, y, nullptr, nullptr, nullptr, st);
+}
+
+inline bool q_tma_ok(const int8_t *q, int64_t K) { return (K % 16) == 0 && aligned(q, 16); }
+
 }  // namespace
 }  // namespace bitnet
 
@@ -433,8 +570,10 @@ BITNET_API int64_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (!sizes_ok(M, N, K)) return -1;
     int64_t need = (int64_t)kAbsmeanMaxBlocks * 8;  // bitnet_absmean partials
     if (M > 0 && N > 0 && K > 0) {
-        const int64_t g = plan_split(M, N, K).ws_bytes;
+        const int64_t g = plan_gemm(M, N, K, false, false).ws_bytes;
+        const int64_t b = plan_gemm(M, N, K, false, true).ws_bytes;
         if (g > need) need = g;
+        if (b > need) need = b;
     }
     return need;
 }
@@ -509,9 +648,9 @@ BITNET_API int bitnet_w2a8_gemm(const int8_t *q, const uint8_t *packed, int32_t 
     if (M == 0 || N == 0) return BITNET_OK;
     if (y == nullptr || (K > 0 && (q == nullptr || packed == nullptr))) return BITNET_ERR_INVALID_ARG;
     if (!aligned(packed, 16) || !aligned(y, 4)) return BITNET_ERR_ALIGNMENT;
-    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BITNET_ERR_WORKSPACE;
-    if (need > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
+    const GemmPlan p = K > 0 ? plan_gemm(M, N, K, q_tma_ok(q, K), false) : GemmPlan{};
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes)) return BITNET_ERR_WORKSPACE;
+    if (p.ws_bytes > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
     DeviceInfo *dev = nullptr;
     int rc = device_info(&dev);
     if (rc != BITNET_OK) return rc;
@@ -520,7 +659,7 @@ BITNET_API int bitnet_w2a8_gemm(const int8_t *q, const uint8_t *packed, int32_t 
         fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, y, nullptr, nullptr, nullptr, workspace, st);
+    return run_w2a8_gemm(dev, q, packed, y, M, N, K, workspace, p, st);
 }
 
 BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const float *gamma, uint16_t *y, int64_t M,
@@ -530,9 +669,9 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     if (y == nullptr || gamma == nullptr || (K > 0 && (x == nullptr || packed == nullptr)))
         return BITNET_ERR_INVALID_ARG;
     if (!aligned(x, 2) || !aligned(packed, 16) || !aligned(y, 2) || !aligned(gamma, 4)) return BITNET_ERR_ALIGNMENT;
-    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BITNET_ERR_WORKSPACE;
-    if (need > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
+    const GemmPlan p = K > 0 ? plan_gemm(M, N, K, false, true) : GemmPlan{};
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes)) return BITNET_ERR_WORKSPACE;
+    if (p.ws_bytes > 0 && !aligned(workspace, 256)) return BITNET_ERR_ALIGNMENT;
     DeviceInfo *dev = nullptr;
     int rc = device_info(&dev);
     if (rc != BITNET_OK) return rc;
@@ -541,8 +680,15 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    // activations are quantised per token inside the GEMV: one launch
-    return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
+    if (p.path == kPathGemv)  // activations quantised per token inside the GEMV: one launch
+        return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
+    // quantise into K_pad-strided rows (zero-padded), then the tensor-core GEMM with the bf16 epilogue
+    const int64_t ldq = k_pad(K);
+    int8_t *q = static_cast<int8_t *>(workspace);
+    float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * ldq, 256));
+    quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, ldq, true, s, nullptr);
+    if ((rc = launched()) != BITNET_OK) return rc;
+    return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, st);
 }
 
 BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M, int64_t N,
@@ -551,8 +697,8 @@ BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, 
     if (M == 0 || N == 0) return BITNET_OK;
     if (y == nullptr || (K > 0 && (q == nullptr || packed == nullptr))) return BITNET_ERR_INVALID_ARG;
     if (!aligned(packed, 16) || !aligned(y, 4)) return BITNET_ERR_ALIGNMENT;
-    const int64_t need = K > 0 ? plan_split(M, N, K).ws_bytes : 0;
-    if (need > (int64_t)BITNET_NOALLOC_SCRATCH_BYTES) return BITNET_ERR_WORKSPACE;
+    const GemmPlan p = K > 0 ? plan_gemm(M, N, K, q_tma_ok(q, K), false) : GemmPlan{};
+    if (p.ws_bytes > (int64_t)BITNET_NOALLOC_SCRATCH_BYTES) return BITNET_ERR_WORKSPACE;
     DeviceInfo *dev = nullptr;
     int rc = device_info(&dev);
     if (rc != BITNET_OK) return rc;
@@ -563,7 +709,7 @@ BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, 
         fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, y, nullptr, nullptr, nullptr, scratch, st);
+    return run_w2a8_gemm(dev, q, packed, y, M, N, K, scratch, p, st);
 }
 
 BITNET_API int bitnet_get_device_error(void *stream) {

@@ -1,0 +1,97 @@
+"""Parity of the tcgen05 tensor-core GEMM (M > 1) with the oracle.
+
+Ragged shapes (M, N not multiples of the tile, K not a multiple of the
+128-byte stage or of 16, which makes the library repack the activations), every
+tile width (forced in child processes through BITNET_GEMV_TUNE, read once per
+process), int32 and BitLinear bf16 outputs.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+import ternary_weight_bit_w2a8_b200 as bn
+from conftest import ROOT
+from ternary_weight_bit_w2a8_b200 import synth
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from ternary_weight_bit_w2a8_b200 import build
+    build.build()
+    yield
+    torch.cuda.synchronize()
+    assert bn.bitnet_get_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 1, 128), (2, 16, 128), (127, 100, 256), (129, 257, 384), (255, 1000, 1040),
+                                   (130, 300, 200), (64, 513, 2560), (300, 96, 999)])
+def test_tc_gemm_ragged_exact(M, N, K):
+    q, w = synth.uniform_int8_ternary(N, K, seed=M + N + K, M=M)
+    q[0, :] = -128  # the int8 extreme in one token
+    y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
+    assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w))
+
+
+def test_tc_gemm_misaligned_activation_rows():
+    # rows of q start at odd offsets: the library repacks them into a workspace
+    M, N, K = 5, 200, 777
+    q, w = synth.uniform_int8_ternary(N, K, seed=3, M=M)
+    base = torch.zeros(M * K + 1, dtype=torch.int8, device="cuda")
+    qd = base[1:].view(M, K)
+    qd.copy_(torch.from_numpy(q))
+    y = bn.bitnet_w2a8_gemm(qd, bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
+    assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w))
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 33, 300), (129, 200, 2560)])
+def test_tc_bitlinear(M, N, K):
+    x, W = synth.bitlinear_inputs(M, N, K, seed=1)
+    g = oracle.absmean(W)
+    wt = oracle.ternarize(W, g)
+    y = bn.bitnet_bitlinear(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16),
+                            bn.bitnet_pack_weights(torch.from_numpy(wt).cuda()),
+                            torch.tensor([float(g)], dtype=torch.float32, device="cuda"), N)
+    y_ref = oracle.bitlinear(x, wt, g)[0]
+    yf = y.float().cpu().numpy().astype(np.float64)
+    err = np.abs(yf - y_ref)
+    assert np.where(np.abs(y_ref) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(y_ref)).all()
+
+
+CHILD = r"""
+import json, sys
+import numpy as np, torch
+sys.path.insert(0, ROOT)
+import oracle
+import ternary_weight_bit_w2a8_b200 as bn
+from ternary_weight_bit_w2a8_b200 import synth
+out = {}
+for (M, N, K) in [(130, 300, 1000), (256, 520, 2560), (3, 1000, 384)]:
+    q, w = synth.uniform_int8_ternary(N, K, seed=M * N + K, M=M)
+    y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
+    out[f"{M}x{N}x{K}"] = bool(np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w)))
+torch.cuda.synchronize()
+out["device_error"] = bn.bitnet_get_device_error()
+print(json.dumps(out))
+"""
+
+
+@pytest.mark.parametrize("tile", [1, 2, 3, 4])  # BN = 256, 128, 96, 64
+def test_tc_every_tile_width(tile):
+    env = dict(os.environ)
+    env["BITNET_GEMV_TUNE"] = f"0,-{tile},0,0,-1,0,-1"
+    r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + CHILD], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert res.pop("device_error") == 0
+    assert all(res.values()), res

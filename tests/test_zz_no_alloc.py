@@ -34,11 +34,11 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
         pytest.skip("no CUDA device")
     lib = bn.lib()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    # (2, 640, 131072) and (2, 64, 65536) split K and keep int32 partials in the
-    # scratch array; for the first, the partials alone exceed the 8 KiB that
-    # bitnet_workspace_bytes reserves for other entry points
-    cases = [(2, 640, 131072), (2, 64, 65536), (1, 300, 2560), (3, 129, 1000), (1, 7, 100)]
-    assert lib.bitnet_workspace_bytes(2, 640, 131072) > 8192
+    # these use the scratch array: (1, 640, 131072) splits K (its activations do
+    # not fit one CTA's shared memory) and keeps int32 partials there; (3, 129,
+    # 1000) and (2, 64, 999) have K not a multiple of 16, so their activations
+    # are repacked there for the tensor-core path; the others need none
+    cases = [(1, 640, 131072), (3, 129, 1000), (2, 64, 999), (1, 300, 2560), (5, 96, 2560), (1, 7, 100)]
     for (M, N, K) in cases:
         for call in range(2):
             q, w = synth.uniform_int8_ternary(N, K, seed=1000 * call + M + N, M=M)
