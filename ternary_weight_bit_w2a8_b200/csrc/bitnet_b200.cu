@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -406,7 +407,7 @@ int noalloc_scratch(void **out) {
 
 // ------------------------------------------------------------------ tcgen05 GEMM (M > 1)
 constexpr int kTcBNs[4] = {256, 128, 96, 64};
-using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmTcArgs);
+using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
 TcKernel tc_kernel_for(int bn_idx, bool bf16, size_t *smem) {
     static const TcKernel k[8] = {gemm_w2a8_tc_kernel<256, false>, gemm_w2a8_tc_kernel<128, false>,
@@ -464,9 +465,27 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         const cuuint32_t box[2] = {32u, (cuuint32_t)BN};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
-                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITNET_ERR_CUDA;
+    }
+    // outputs: 32-row boxes of 128 bytes per row, stored through TMA when the
+    // rows are 16-byte strided and the base 16-byte aligned
+    CUtensorMap ymap;
+    memset(&ymap, 0, sizeof(ymap));
+    const int esize = bf16 ? 2 : 4;
+    void *ybase = bf16 ? static_cast<void *>(y_bf16) : static_cast<void *>(y_i32);
+    int tma_store = ((N * esize) % 16 == 0) && aligned(ybase, 16);
+    if (tma_store) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)(N * esize)};
+        const cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 32u};
+        const cuuint32_t es[2] = {1, 1};
+        if (tensor_map_encoder()(&ymap, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_INT32, 2,
+                                 ybase, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            tma_store = 0;
     }
     GemmTcArgs a{};
     a.M = M;
@@ -477,8 +496,9 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.y_bf16 = y_bf16;
     a.s_act = s_act;
     a.gamma = gamma;
+    a.tma_store = tma_store;
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)ceil_div(M, kTcBM));
-    return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, a));
+    return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, ymap, a));
 }
 
 // Copies int8 activations [M, K] into rows of K_pad bytes, zero-padded, so the

@@ -22,8 +22,10 @@
 //     comes out of the tensor core, with no extra pass over q.
 //     tcgen05.commit on a per-stage mbarrier releases the stage.
 //   - After the last stage, warps 2..5 read the accumulators (tcgen05.ld, one
-//     row per thread), subtract the row sum and store int32, or scale by
-//     gamma / s_m and store bf16.
+//     row per thread), subtract the row sum and either keep int32 or scale by
+//     gamma / s_m to bf16, stage 32-row boxes in the freed operand ring with
+//     the 128-byte swizzle and write them with TMA stores (full lines); direct
+//     stores are the fallback when the output rows are not 16-byte strided.
 //   - Every mbarrier wait is bounded in time; a role that gives up records
 //     BITNET_ERR_DEVICE_TIMEOUT and raises a shared abort flag that stops the
 //     others; all roles then drain what they issued (bounded) and tensor
@@ -48,6 +50,7 @@ constexpr int kTcOnesRows = 16;
 struct GemmTcArgs {
     int64_t M, N, K;
     int nk;                 // k stages: K_pad / 128
+    int tma_store;          // 1: outputs leave through TMA stores of swizzled boxes (y rows 16-byte strided)
     int32_t *y_i32;         // [M, N] int32 result
     uint16_t *y_bf16;       // [M, N] bf16 result (BitLinear)
     const float *s_act;     // [M] activation scales (BitLinear)
@@ -135,10 +138,25 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
     tma_load_box(dst, map, x, y, bar);
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, const void *src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+                 "r"(y), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until at most n committed bulk stores still read shared memory.
+template <int n>
+__device__ __forceinline__ void tma_store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory");
+}
+
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int BN, bool BF16_OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
-                        const GemmTcArgs a) {
+                        const __grid_constant__ CUtensorMap ymap, const GemmTcArgs a) {
     using L = TcSmem<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -249,8 +267,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint8_t *bs = sm + L::kB + s * L::kBStage;
 #pragma unroll
             for (int n = t; n < BN; n += 128) {
-                const uint4 p0 = *reinterpret_cast<const uint4 *>(ps + n * 32);
-                const uint4 p1 = *reinterpret_cast<const uint4 *>(ps + n * 32 + 16);
+                // the packed tile arrives with the 32-byte swizzle: 16-byte half h of
+                // row n sits at n * 32 + ((h ^ ((n >> 2) & 1)) * 16)
+                const int sw = (n >> 2) & 1;
+                const uint4 p0 = *reinterpret_cast<const uint4 *>(ps + n * 32 + (sw << 4));
+                const uint4 p1 = *reinterpret_cast<const uint4 *>(ps + n * 32 + ((sw ^ 1) << 4));
                 const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
                 uint8_t *row = bs + n * kTcBK;
 #pragma unroll
@@ -277,25 +298,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float f = 0.0f;
             if (BF16_OUT && m < a.M) f = __fdiv_rn(*a.gamma, a.s_act[m]);
             pdl_wait();  // the outputs may still be read by the previous kernel
+            if (a.tma_store) {
+                // Stage 32-row boxes (128 bytes per row: 32 int32 or 64 bf16 values)
+                // in the freed activation ring with the 128-byte swizzle (thread =
+                // row, conflict-free), two buffers per warp, and store each box
+                // with one TMA store; the TMA unit clips rows >= M and columns >= N.
+                constexpr int kCols = BF16_OUT ? 64 : 32;
+                uint8_t *wbuf = sm + L::kA + quarter * 2 * 4096;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                tmem_ld16(tbase + c, v);
-                if (m < a.M) {
-                    const int64_t nb = n0 + c;
+                for (int c = 0, it = 0; c < BN; c += kCols, ++it) {
+                    uint8_t *buf = wbuf + (it & 1) * 4096;
+                    if (it >= 2) {
+                        if (lane == 0) tma_store_wait_read<1>();
+                        __syncwarp();
+                    }
+                    uint32_t packed_row[32];
                     if (BF16_OUT) {
-                        uint16_t *dst = a.y_bf16 + m * a.N + nb;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (nb + i < a.N) dst[i] = float_to_bf16_bits_rn(__fmul_rn((float)((int)v[i] - rowsum), f));
+                        for (int h = 0; h < 4; ++h) {
+                            tmem_ld16(tbase + c + 16 * h, v);
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2) {
+                                const uint32_t lo = float_to_bf16_bits_rn(__fmul_rn((float)((int)v[i] - rowsum), f));
+                                const uint32_t hi = float_to_bf16_bits_rn(__fmul_rn((float)((int)v[i + 1] - rowsum), f));
+                                packed_row[8 * h + i / 2] = lo | (hi << 16);
+                            }
+                        }
                     } else {
-                        int32_t *dst = a.y_i32 + m * a.N + nb;
-                        if (nb + 16 <= a.N && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
 #pragma unroll
-                            for (int i = 0; i < 16; i += 4)
-                                *reinterpret_cast<int4 *>(dst + i) =
-                                    make_int4((int)v[i] - rowsum, (int)v[i + 1] - rowsum, (int)v[i + 2] - rowsum,
-                                              (int)v[i + 3] - rowsum);
+                        for (int h = 0; h < 2; ++h) {
+                            tmem_ld16(tbase + c + 16 * h, v);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) packed_row[16 * h + i] = (uint32_t)((int)v[i] - rowsum);
+                        }
+                    }
+                    uint8_t *rowp = buf + lane * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4 *>(rowp + ((j ^ (lane & 7)) << 4)) =
+                            make_uint4(packed_row[4 * j], packed_row[4 * j + 1], packed_row[4 * j + 2],
+                                       packed_row[4 * j + 3]);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&ymap, (int)(n0 + c), (int)(m0 + quarter * 32), buf);
+                }
+                if (lane == 0) tma_store_wait_all();
+                __syncwarp();
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    tmem_ld16(tbase + c, v);
+                    if (m < a.M) {
+                        const int64_t nb = n0 + c;
+                        if (BF16_OUT) {
+                            uint16_t *dst = a.y_bf16 + m * a.N + nb;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (nb + i < a.N)
+                                    dst[i] = float_to_bf16_bits_rn(__fmul_rn((float)((int)v[i] - rowsum), f));
                         } else {
+                            int32_t *dst = a.y_i32 + m * a.N + nb;
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
                                 if (nb + i < a.N) dst[i] = (int)v[i] - rowsum;
