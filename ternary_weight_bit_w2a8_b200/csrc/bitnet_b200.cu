@@ -428,12 +428,37 @@ int tc_bn_index(int64_t M, int64_t N, int sm_count) {
     return 3;
 }
 
+// Tile width and K-split of the tensor-core GEMM.  Computed for the B200's
+// 148 SMs whatever the device, so the workspace a shape needs is fixed.
+struct TcPlan {
+    int bn_idx, S, sps;
+};
+
+TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
+    constexpr int kRefSMs = 148;
+    TcPlan p{};
+    const GemvTune &tn = gemv_tune();
+    p.bn_idx = tc_bn_index(M, N, kRefSMs);
+    if (tn.R < 0 && -tn.R <= 4) p.bn_idx = -tn.R - 1;  // tuning override: R = -1..-4 picks the tile width
+    const int nk = (int)(k_pad(K) / kTcBK);
+    const int64_t tiles = ceil_div(M, kTcBM) * ceil_div(N, kTcBNs[p.bn_idx]);
+    int S = 1;
+    if (tiles * 2 <= kRefSMs && nk >= 8) {
+        S = (int)(kRefSMs / tiles);
+        if (S > nk / 4) S = nk / 4;
+        if (S < 1) S = 1;
+    }
+    if (tn.S > 0) S = tn.S < nk ? tn.S : nk;  // tuning override
+    p.sps = (int)ceil_div(nk, S);
+    p.S = (int)ceil_div(nk, p.sps);
+    return p;
+}
+
+// reduce: add int32 results into y_i32 (which the caller has zeroed).
 int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t *packed, int64_t M, int64_t N,
                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
-                   cudaStream_t st) {
-    const GemvTune &tn = gemv_tune();
-    int bi = tc_bn_index(M, N, dev->sm_count);
-    if (tn.R < 0 && -tn.R <= 4) bi = -tn.R - 1;  // tuning override: R = -1..-4 picks the tile width
+                   const TcPlan &tp, int reduce, cudaStream_t st) {
+    const int bi = tp.bn_idx;
     const int BN = kTcBNs[bi];
     const bool bf16 = y_bf16 != nullptr;
     size_t smem = 0;
@@ -497,7 +522,9 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.s_act = s_act;
     a.gamma = gamma;
     a.tma_store = tma_store;
-    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)ceil_div(M, kTcBM));
+    a.sps = tp.sps;
+    a.reduce = reduce;
+    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)ceil_div(M, kTcBM), (unsigned)tp.S);
     return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, ymap, a));
 }
 
@@ -512,6 +539,20 @@ __global__ void __launch_bounds__(kThreads) repack_q_kernel(const int8_t *__rest
     }
 }
 
+// BitLinear epilogue after a K-split: y = bf16_rne(acc * (gamma / s_m)), the
+// same fp32 operations as the GEMM's own epilogue.
+__global__ void __launch_bounds__(kThreads) rescale_bf16_kernel(const int32_t *__restrict__ acc, int64_t M, int64_t N,
+                                                                const float *__restrict__ s, const float *__restrict__ gamma,
+                                                                uint16_t *__restrict__ y) {
+    pdl_wait();
+    const float g = *gamma;
+    const int64_t total = M * N;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += (int64_t)gridDim.x * kThreads) {
+        const float f = __fdiv_rn(g, s[i / N]);
+        y[i] = float_to_bf16_bits_rn(__fmul_rn((float)acc[i], f));
+    }
+}
+
 // ------------------------------------------------------------------ dispatch
 // One plan for every caller of the contraction, so the path taken and the
 // scratch it needs always agree.
@@ -520,15 +561,18 @@ struct GemmPlan {
     int path;
     bool repack;       // int8 activations copied to K_pad-strided rows first
     int64_t ws_bytes;
+    TcPlan tc;
 };
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinear) {
     GemmPlan p{};
     if (M >= 2 && K >= kTcBK && tensor_map_encoder() != nullptr) {
         p.path = kPathTc;
+        p.tc = tc_plan(M, N, K);
         const int64_t qbytes = round_up(M * k_pad(K), 256);
         if (bitlinear) {
-            p.ws_bytes = qbytes + round_up(M * 4, 256);
+            // quantised activations, scales and, for a K-split, int32 sums
+            p.ws_bytes = qbytes + round_up(M * 4, 256) + (p.tc.S > 1 ? round_up(M * N * 4, 256) : 0);
         } else {
             p.repack = !q_tma_ok;
             p.ws_bytes = p.repack ? qbytes : 0;
@@ -554,7 +598,12 @@ int run_w2a8_gemm(DeviceInfo *dev, const int8_t *q, const uint8_t *packed, int32
         if (rc != BITNET_OK) return rc;
         qa = qp;
     }
-    return launch_gemm_tc(dev, qa, lda, packed, M, N, K, y, nullptr, nullptr, nullptr, st);
+    if (p.tc.S > 1) {  // K-split: the splits add into a zeroed output
+        fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
+        const int rc = launched();
+        if (rc != BITNET_OK) return rc;
+    }
+    return launch_gemm_tc(dev, qa, lda, packed, M, N, K, y, nullptr, nullptr, nullptr, p.tc, p.tc.S > 1, st);
 }
 
 inline bool q_tma_ok(const int8_t *q, int64_t K) { return (K % 16) == 0 && aligned(q, 16); }
@@ -708,7 +757,15 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * ldq, 256));
     quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, ldq, true, s, nullptr);
     if ((rc = launched()) != BITNET_OK) return rc;
-    return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, st);
+    if (p.tc.S == 1) return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, p.tc, 0, st);
+    // K-split: int32 sums in the workspace, then the rescale to bf16
+    int32_t *acc = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(s) + round_up(M * 4, 256));
+    fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(acc, M * N, 0);
+    if ((rc = launched()) != BITNET_OK) return rc;
+    if ((rc = launch_gemm_tc(dev, q, ldq, packed, M, N, K, acc, nullptr, nullptr, nullptr, p.tc, 1, st)) != BITNET_OK)
+        return rc;
+    return launched(launch_pdl(rescale_bf16_kernel, dim3(grid_for(M * N, kThreads * 4, dev->sm_count)),
+                               dim3(kThreads), (size_t)0, st, (const int32_t *)acc, M, N, (const float *)s, gamma, y));
 }
 
 BITNET_API int bitnet_w2a8_gemm_noalloc(const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M, int64_t N,

@@ -26,6 +26,10 @@
 //     gamma / s_m to bf16, stage 32-row boxes in the freed operand ring with
 //     the 128-byte swizzle and write them with TMA stores (full lines); direct
 //     stores are the fallback when the output rows are not 16-byte strided.
+//   - Split-K (gridDim.z > 1, for problems with fewer tiles than SMs): each
+//     split covers a range of k stages, subtracts its own share of the row
+//     sums, and adds its int32 results into a zeroed output with TMA
+//     reduce-add stores (integer adds: exact and order-free).
 //   - Every mbarrier wait is bounded in time; a role that gives up records
 //     BITNET_ERR_DEVICE_TIMEOUT and raises a shared abort flag that stops the
 //     others; all roles then drain what they issued (bounded) and tensor
@@ -51,6 +55,8 @@ struct GemmTcArgs {
     int64_t M, N, K;
     int nk;                 // k stages: K_pad / 128
     int tma_store;          // 1: outputs leave through TMA stores of swizzled boxes (y rows 16-byte strided)
+    int sps;                // k stages per split (split-K over gridDim.z)
+    int reduce;             // 1: add int32 results into the (zeroed) output instead of storing them
     int32_t *y_i32;         // [M, N] int32 result
     uint16_t *y_bf16;       // [M, N] bf16 result (BitLinear)
     const float *s_act;     // [M] activation scales (BitLinear)
@@ -153,6 +159,14 @@ __device__ __forceinline__ void tma_store_wait_read() {
 
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Element-wise add of a shared-memory box into global memory (exact for s32).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x, int y, const void *src) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
 template <int BN, bool BF16_OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
@@ -171,7 +185,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n0 = (int64_t)blockIdx.x * BN, m0 = (int64_t)blockIdx.y * kTcBM;
-    const int nk = a.nk;
+    const int kbase = blockIdx.z * a.sps;  // this split's first k stage
+    const int nk = min(a.sps, a.nk - kbase);
 
     // ---- set-up: barriers, the ones tile, tensor memory
     if (threadIdx.x == 0) {
@@ -212,8 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (kb >= kTcStages && !tc_wait(&mma_done[s], (uint32_t)((kb / kTcStages) - 1) & 1u, abort_flag))
                     break;
                 mbar_arrive_expect_tx(&tma_full[s], kTcAStageBytes + L::kPStage);
-                tma_load_2d(sm + L::kA + s * kTcAStageBytes, &amap, kb * kTcBK, (int)m0, &tma_full[s]);
-                tma_load_2d(sm + L::kP + s * L::kPStage, &pmap, kb * 32, (int)n0, &tma_full[s]);
+                tma_load_2d(sm + L::kA + s * kTcAStageBytes, &amap, (kbase + kb) * kTcBK, (int)m0, &tma_full[s]);
+                tma_load_2d(sm + L::kP + s * L::kPStage, &pmap, (kbase + kb) * 32, (int)n0, &tma_full[s]);
                 issued = kb + 1;
             }
             // make sure no copy is still landing in shared memory when the CTA leaves
@@ -340,7 +355,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                        packed_row[4 * j + 3]);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&ymap, (int)(n0 + c), (int)(m0 + quarter * 32), buf);
+                    if (lane == 0) {
+                        if (a.reduce)
+                            tma_reduce_add_2d(&ymap, (int)(n0 + c), (int)(m0 + quarter * 32), buf);
+                        else
+                            tma_store_2d(&ymap, (int)(n0 + c), (int)(m0 + quarter * 32), buf);
+                    }
                 }
                 if (lane == 0) tma_store_wait_all();
                 __syncwarp();
@@ -359,8 +379,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         } else {
                             int32_t *dst = a.y_i32 + m * a.N + nb;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (nb + i < a.N) dst[i] = (int)v[i] - rowsum;
+                            for (int i = 0; i < 16; ++i) {
+                                if (nb + i < a.N) {
+                                    if (a.reduce)
+                                        atomicAdd(dst + i, (int)v[i] - rowsum);
+                                    else
+                                        dst[i] = (int)v[i] - rowsum;
+                                }
+                            }
                         }
                     }
                 }
