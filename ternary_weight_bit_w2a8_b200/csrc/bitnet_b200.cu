@@ -36,7 +36,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[6] = {0, 0, 0, 0, 0, 0};  // dynamic shared memory opted into by each TMA GEMV
+    size_t tma_max_dyn[10] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[8] = {false, false, false, false, false, false, false, false};
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -204,32 +204,25 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 
 // TMA GEMV variants: (warps per CTA, boxes in flight per warp)
-constexpr int kTmaCfg[3][2] = {{8, 4}, {12, 3}, {16, 2}};
+constexpr int kTmaNumCfg = 5;
+constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
 TmaKernel tma_kernel_for(int xmode, int cfg) {
-    static const TmaKernel table[6] = {gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 12, 3>, gemv_tma_kernel<0, 16, 2>,
-                                       gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 12, 3>, gemv_tma_kernel<1, 16, 2>};
-    return table[xmode * 3 + cfg];
+    static const TmaKernel table[2 * kTmaNumCfg] = {
+        gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 12, 3>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 2>,
+        gemv_tma_kernel<0, 4, 4>, gemv_tma_kernel<1, 8, 4>,  gemv_tma_kernel<1, 12, 3>, gemv_tma_kernel<1, 16, 2>,
+        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 4, 4>};
+    return table[xmode * kTmaNumCfg + cfg];
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
 size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    size_t &slot = dev->tma_max_dyn[xmode * 3 + cfg];
+    size_t &slot = dev->tma_max_dyn[xmode * kTmaNumCfg + cfg];
     if (slot == 0) {
         TmaKernel kern = tma_kernel_for(xmode, cfg);
-    // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
-    // makes one wait run out, exercising the device-timeout path
-    static std::atomic<int> stall_once{-1};
-    if (stall_once.load() == -1) {
-        const char *e = getenv("BITNET_TEST_STALL");
-        int expect = -1;
-        stall_once.compare_exchange_strong(expect, (e != nullptr && e[0] == '1') ? 1 : 0);
-    }
-    int one = 1;
-    const int test_stall = stall_once.compare_exchange_strong(one, 0) ? 1 : 0;
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -239,32 +232,70 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
     return slot;
 }
 
-// Shared memory the TMA GEMV needs for this shape on this device, or 0 if it
-// does not apply (then the register-streaming GEMV runs).
-size_t tma_plan(DeviceInfo *dev, int xmode, int64_t M, int64_t N, int64_t K, int *cfg, int *slices, int *max_blocks,
-                int *grid) {
+// Plan of the M = 1 TMA GEMV, from the shape and B200 reference figures only
+// (148 SMs, 228 KB of shared memory per SM), so that the workspace a shape
+// needs does not depend on the device that runs it.
+struct TmaPlan {
+    bool use;
+    int cfg, slices, max_blocks, grid, max_parts;
+    int64_t ipc;       // > 0: split mode
+    size_t smem;
+    int64_t ws_bytes;  // split mode: int32 parts and the BitLinear scale
+};
+
+TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
+    constexpr int kRefSMs = 148;
+    constexpr size_t kRefSmemPerSM = 233472, kRefCtaReserve = 1024, kRefSmemOptin = 232448;
+    TmaPlan p{};
     const int tune = gemv_tune().tma;
-    if (M != 1 || tune == 0 || K < kTmaSliceK) return 0;
+    if (M != 1 || tune == 0 || K < kTmaSliceK || N < 1) return p;
     const int64_t row_bytes = packed_row_bytes(K);
     const int64_t nblocks = ceil_div(N, kTmaRows);
-    const int64_t g = nblocks < dev->sm_count ? nblocks : dev->sm_count;
-    *slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
-    *max_blocks = (int)ceil_div(nblocks, g);
-    *grid = (int)g;
-    // measured on B200: more warps with fewer boxes each win once every SM
-    // has several row blocks; long rows prefer 12 x 3; small problems 8 x 4
-    if (tune >= 1 && tune <= 3)
-        *cfg = tune - 1;
+    p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
+    // variant (measured on B200 over the sweep and large shapes): 16 warps x 2
+    // boxes in general, 12 x 3 for rows of K >= 16384, 8 x 4 below 3 MB
+    if (tune >= 1 && tune <= kTmaNumCfg)
+        p.cfg = tune - 1;
     else
-        *cfg = nblocks >= 4 * (int64_t)dev->sm_count ? 2 : (*slices >= 32 ? 1 : 0);
-    const size_t smem = gemv_tma_smem_bytes(kTmaCfg[*cfg][0], kTmaCfg[*cfg][1], *slices, *max_blocks);
-    if (tensor_map_encoder() == nullptr || smem > tma_max_dynamic_smem(dev, xmode, *cfg)) return 0;
-    return smem;
+        p.cfg = N * row_bytes < (3ll << 20) ? 0 : (p.slices >= 32 ? 1 : 2);
+    const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
+    // resident CTAs per SM for the block-strided layout (accumulator slots are small)
+    const size_t base_smem = gemv_tma_smem_bytes(W, NS, p.slices, 1);
+    int per_sm = (int)(kRefSmemPerSM / (base_smem + kRefCtaReserve));
+    if (per_sm > 2048 / (W * 32)) per_sm = 2048 / (W * 32);
+    if (per_sm < 1) return p;
+    const int64_t gmax = (int64_t)kRefSMs * per_sm;
+    // split mode when whole row blocks per CTA would leave CTAs idle or uneven
+    // (more than 15 % above the mean), for problems large enough to pay the
+    // fixup launch (>= 4 MB of weights)
+    const int64_t g_strided = nblocks < gmax ? nblocks : gmax;
+    const double mean = (double)nblocks / (double)gmax, worst = (double)ceil_div(nblocks, g_strided);
+    // (measured on B200: the fixup launch costs more than the balance gains for
+    // every shape tried, so split mode is used only when asked for)
+    (void)mean;
+    (void)worst;
+    const bool want_split = gemv_tune().S == 1;
+    if (want_split) {
+        const int64_t items = nblocks * p.slices;
+        p.ipc = ceil_div(items, gmax);
+        p.grid = (int)ceil_div(items, p.ipc);
+        p.max_blocks = (int)(ceil_div(p.ipc, p.slices) + 1);
+        p.max_parts = (int)(ceil_div(p.slices, p.ipc) + 1);
+        p.ws_bytes = round_up(nblocks * p.max_parts * kTmaRows * 4, 256) + 256;
+    } else {
+        p.grid = (int)g_strided;
+        p.max_blocks = (int)ceil_div(nblocks, g_strided);
+    }
+    p.smem = gemv_tma_smem_bytes(W, NS, p.slices, p.max_blocks);
+    if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
+    p.use = true;
+    return p;
 }
 
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t N,
-                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, int cfg, int slices,
-                    int max_blocks, int grid, size_t smem, cudaStream_t st) {
+                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const TmaPlan &tp, void *ws,
+                    cudaStream_t st) {
+    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg)) return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
     const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
@@ -275,7 +306,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
                              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return BITNET_ERR_CUDA;
-    TmaKernel kern = tma_kernel_for(xmode, cfg);
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg);
     // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
     // makes one wait run out, exercising the device-timeout path
     static std::atomic<int> stall_once{-1};
@@ -291,15 +322,23 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.x = x;
     a.N = N;
     a.K = K;
-    a.slices = slices;
+    a.slices = tp.slices;
     a.blk_begin = 0;
     a.nblocks = ceil_div(N, kTmaRows);
-    a.max_blocks_cta = max_blocks;
+    a.max_blocks_cta = tp.max_blocks;
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
     a.test_stall = test_stall;
-    return launched(launch_pdl(kern, dim3(grid), dim3(kTmaCfg[cfg][0] * 32), smem, st, map, a));
+    a.ipc = tp.ipc;
+    a.max_parts = tp.max_parts;
+    if (tp.ipc > 0) {
+        a.parts = static_cast<int32_t *>(ws);
+        a.s_out = reinterpret_cast<float *>(static_cast<char *>(ws) + tp.ws_bytes - 256);
+    }
+    int rc = launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
+    if (rc != BITNET_OK || tp.ipc == 0) return rc;
+    return launched(launch_pdl(gemv_tma_fixup_kernel, dim3(grid_for(N, 256, dev->sm_count)), dim3(256), (size_t)0, st, a));
 }
 
 // xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
@@ -308,11 +347,8 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
                 const uint8_t *packed, int64_t M, int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16,
                 const float *s_act, const float *gamma, void *ws, cudaStream_t st) {
     {
-        int cfg = 0, slices = 0, max_blocks = 0, grid = 0;
-        const size_t smem = tma_plan(dev, xmode, M, N, K, &cfg, &slices, &max_blocks, &grid);
-        if (smem > 0 && ldq == K)
-            return launch_gemv_tma(dev, xmode, q, x, packed, N, K, y_i32, y_bf16, gamma, cfg, slices, max_blocks,
-                                   grid, smem, st);
+        const TmaPlan tp = tma_plan(M, N, K);
+        if (tp.use) return launch_gemv_tma(dev, xmode, q, x, packed, N, K, y_i32, y_bf16, gamma, tp, ws, st);
     }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();
@@ -458,6 +494,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
 int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t *packed, int64_t M, int64_t N,
                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
                    const TcPlan &tp, int reduce, cudaStream_t st) {
+    if (tensor_map_encoder() == nullptr) return BITNET_ERR_CUDA;
     const int bi = tp.bn_idx;
     const int BN = kTcBNs[bi];
     const bool bf16 = y_bf16 != nullptr;
@@ -566,7 +603,7 @@ struct GemmPlan {
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinear) {
     GemmPlan p{};
-    if (M >= 2 && K >= kTcBK && tensor_map_encoder() != nullptr) {
+    if (M >= 2 && K >= kTcBK) {
         p.path = kPathTc;
         p.tc = tc_plan(M, N, K);
         const int64_t qbytes = round_up(M * k_pad(K), 256);
@@ -579,7 +616,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
         }
     } else {
         p.path = kPathGemv;
-        p.ws_bytes = plan_split(M, N, K).ws_bytes;
+        const TmaPlan tp = tma_plan(M, N, K);
+        p.ws_bytes = tp.use ? tp.ws_bytes : plan_split(M, N, K).ws_bytes;
     }
     return p;
 }

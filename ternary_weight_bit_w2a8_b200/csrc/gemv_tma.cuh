@@ -51,6 +51,13 @@ struct GemvTmaArgs {
     int64_t blk_begin;    // first row block of this launch
     int64_t nblocks;      // row blocks of this launch
     int max_blocks_cta;   // accumulator slots per CTA
+    // split mode (ipc > 0): CTA c takes items [c * ipc, (c + 1) * ipc) of the
+    // global (row block, slice) list and writes one int32 part per row block it
+    // touches to parts[block][c - first CTA of the block][32]
+    int64_t ipc;
+    int max_parts;        // parts per row block
+    int32_t *parts;
+    float *s_out;         // BitLinear split mode: the activation scale, for the fixup
     int32_t *y_i32;       // [M, N] int32 result
     uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
     const float *gamma;   // weight scale (BitLinear)
@@ -61,7 +68,8 @@ struct GemvTmaArgs {
 // activations, per-row-block accumulators and counters, mbarriers.
 __host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta) {
     return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes + (size_t)slices * kTmaSliceK +
-           (size_t)max_blocks_cta * kTmaRows * 4 + (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8;
+           (size_t)max_blocks_cta * kTmaRows * 4 + (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 +
+           (size_t)slices * 4;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -112,10 +120,21 @@ __device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *map, 
         : "memory");
 }
 
-// Linear staging of int8 activations: qlin[k] = q[k] for k < K, 0 up to kq.
-__device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, const int8_t *qrow, int64_t K, int64_t kq) {
+// Adds up the 16-byte piece p of this lane into its K-slice's activation sum:
+// a warp stages 32 consecutive pieces (p = 32 w' + lane), exactly one slice of
+// 512 k, so one warp reduction gives the slice's sum.
+__device__ __forceinline__ void slice_sum(int *qslice, int64_t p, const uint4 &v) {
+    const int t = group_sum<32>(byte_sum(v, 0));
+    if ((threadIdx.x & 31) == 0) qslice[p >> 5] = t;
+}
+
+// Linear staging of int8 activations: qlin[k] = q[k] for k < K, 0 up to kq
+// (kq a multiple of 512), with the sum of every 512-k slice in qslice.
+__device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, int *qslice, const int8_t *qrow, int64_t K,
+                                                int64_t kq) {
     const bool vec = ((reinterpret_cast<uintptr_t>(qrow) & 15) == 0);
-    for (int64_t k0 = (int64_t)threadIdx.x * 16; k0 < kq; k0 += (int64_t)blockDim.x * 16) {
+    for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
+        const int64_t k0 = p * 16;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (vec && k0 + 16 <= K) {
             v = *reinterpret_cast<const uint4 *>(qrow + k0);
@@ -125,13 +144,14 @@ __device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, const int8_t *qrow
             v = make_uint4(w[0], w[1], w[2], w[3]);
         }
         *reinterpret_cast<uint4 *>(qlin + k0) = v;
+        slice_sum(qslice, p, v);
     }
 }
 
 // Linear staging with fused per-token quantisation of bf16 activations (same
-// arithmetic as quant_act_kernel).  Returns the scale.
-__device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, float *red, const uint16_t *xrow, int64_t K,
-                                                 int64_t kq) {
+// arithmetic as quant_act_kernel), slice sums as above.  Returns the scale.
+__device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, float *red, const uint16_t *xrow,
+                                                 int64_t K, int64_t kq) {
     constexpr int kHeld = 4;
     const bool vec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
     const int64_t npieces = ceil_div(K, 16), qpieces = kq / 16;
@@ -159,6 +179,7 @@ __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, float *red, const
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (p < npieces) quant16(held[h][0], held[h][1], sc, v);
             *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
+            slice_sum(qslice, p, v);
         }
     }
     for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < qpieces; p += blockDim.x) {
@@ -169,6 +190,7 @@ __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, float *red, const
             quant16(lo, hi, sc, v);
         }
         *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
+        slice_sum(qslice, p, v);
     }
     return sc;
 }
@@ -185,13 +207,31 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     const int64_t kq = (int64_t)a.slices * kTmaSliceK;
     int *accs = reinterpret_cast<int *>(qlin + kq);
     int *done = accs + a.max_blocks_cta * kTmaRows;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(done + a.max_blocks_cta + ((a.max_blocks_cta & 1) ? 1 : 0));
+    int *qslice = done + a.max_blocks_cta;   // activation sum of each K-slice
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qslice + a.slices + ((a.max_blocks_cta + a.slices) & 1));
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slices = a.slices;
-    const int64_t nb_cta = a.nblocks > blockIdx.x ? ceil_div(a.nblocks - blockIdx.x, gridDim.x) : 0;
-    const int64_t items = nb_cta * slices;
-    // this warp's items: a contiguous range of (row block, slice) pairs
+    const bool split = a.ipc > 0;
+    // this CTA's items, in (row block, slice) order; `bstep` is the distance
+    // between consecutive row blocks of the CTA
+    int64_t cta_begin, items, first_block, bstep;
+    if (split) {
+        const int64_t total = a.nblocks * slices;
+        cta_begin = min(total, (int64_t)blockIdx.x * a.ipc);
+        items = min(total, cta_begin + a.ipc) - cta_begin;
+        first_block = cta_begin / slices;
+        bstep = 1;
+    } else {
+        const int64_t nb_cta = a.nblocks > blockIdx.x ? ceil_div(a.nblocks - blockIdx.x, gridDim.x) : 0;
+        cta_begin = 0;
+        items = nb_cta * slices;
+        first_block = blockIdx.x;
+        bstep = gridDim.x;
+    }
+    const int j0 = (int)(split ? cta_begin - first_block * slices : 0);  // slice of the CTA's first item
+    const int nslots = (int)((j0 + items + slices - 1) / slices);        // row blocks touched
+    // this warp's items: a contiguous range of the CTA's items
     const int64_t ipw = ceil_div(items, W);
     const int64_t it_begin = min(items, warp * ipw);
     const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
@@ -199,21 +239,21 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     uint8_t *myring = ring + warp * NS * kTmaBoxBytes;
 
     if (threadIdx.x < W * NS) mbar_init(&bars[threadIdx.x], 1);
-    for (int64_t i = threadIdx.x; i < nb_cta * kTmaRows; i += blockDim.x) accs[i] = 0;
-    for (int64_t i = threadIdx.x; i < nb_cta; i += blockDim.x) done[i] = 0;
+    for (int i = threadIdx.x; i < nslots * kTmaRows; i += blockDim.x) accs[i] = 0;
+    for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
 
-    // issue cursor (lane 0 only): next item to request
-    int64_t ibl = it_begin / slices;
-    int ij = (int)(it_begin - ibl * slices);
+    // cursor over the warp's items: (slot, slice); row block = first_block + slot * bstep
+    const int64_t p0 = j0 + it_begin;
+    int islot = (int)(p0 / slices), ij = (int)(p0 - (int64_t)(p0 / slices) * slices);
     auto issue_next = [&](int s) {
-        const int64_t row0 = (a.blk_begin + blockIdx.x + ibl * gridDim.x) * kTmaRows;
+        const int64_t row0 = (a.blk_begin + first_block + (int64_t)islot * bstep) * kTmaRows;
         mbar_arrive_expect_tx(&mybar[s], kTmaBoxBytes);
         tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
         if (++ij == slices) {
             ij = 0;
-            ++ibl;
+            ++islot;
         }
     };
     // weights do not depend on the previous kernel: request them before waiting for it
@@ -222,7 +262,7 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
             if (s == 0 && warp == 0 && a.test_stall) {  // skip the request: nothing completes this stage
                 if (++ij == slices) {
                     ij = 0;
-                    ++ibl;
+                    ++islot;
                 }
                 continue;
             }
@@ -234,48 +274,56 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
 
     float sc = 0.0f;
     if (XMODE == 0)
-        stage_qlin_int8(qlin, a.q, a.K, kq);
+        stage_qlin_int8(qlin, qslice, a.q, a.K, kq);
     else
-        sc = stage_qlin_bf16(qlin, red, a.x, a.K, kq);
+        sc = stage_qlin_bf16(qlin, qslice, red, a.x, a.K, kq);
+    if (split && XMODE == 1 && a.s_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.s_out = sc;
     __syncthreads();
-
-    int qsum = 0;
-    for (int64_t p = lane; p < kq / 16; p += 32) qsum = byte_sum(reinterpret_cast<const uint4 *>(qlin)[p], qsum);
-    qsum = group_sum<32>(qsum);
     float f = 0.0f;
-    if (XMODE == 1) f = __fdiv_rn(*a.gamma, sc);
+    if (XMODE == 1 && !split) f = __fdiv_rn(*a.gamma, sc);
 
     int acc[4] = {0, 0, 0, 0};
-    int ncontrib = 0;
-    // folds this warp's partial sums of row block `bl` into shared memory; the
-    // warp completing the block writes its 32 outputs
-    auto flush = [&](int64_t bl) {
-        const int v = acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6);
-        atomicAdd(&accs[bl * kTmaRows + lane], v);
+    int ncontrib = 0, corr = 0;
+    // folds this warp's partial sums of slot `sl` into shared memory; the warp
+    // completing the slot's items writes its 32 results (split mode: its part)
+    auto flush = [&](int sl) {
+        const int v = acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6) - corr;
+        atomicAdd(&accs[sl * kTmaRows + lane], v);
         __threadfence_block();
         __syncwarp();
+        const int64_t blk = first_block + (int64_t)sl * bstep;
+        int expected = slices;
+        if (split) {
+            const int64_t lo = max(cta_begin, blk * slices), hi = min(cta_begin + items, (blk + 1) * slices);
+            expected = (int)(hi - lo);
+        }
         int fin = 0;
-        if (lane == 0) fin = (atomicAdd(&done[bl], ncontrib) + ncontrib == slices);
+        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == expected);
         fin = __shfl_sync(0xffffffffu, fin, 0);
         if (fin) {
             __threadfence_block();
-            const int tot = atomicAdd(&accs[bl * kTmaRows + lane], 0);
-            const int64_t n = (a.blk_begin + blockIdx.x + bl * gridDim.x) * kTmaRows + lane;
-            if (n < a.N) {
-                const int r = tot - qsum;
-                if (XMODE == 1)
-                    a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)r, f));
-                else
-                    a.y_i32[n] = r;
+            const int tot = atomicAdd(&accs[sl * kTmaRows + lane], 0);
+            const int64_t gb = a.blk_begin + blk;
+            if (split) {
+                const int64_t first_cta = (gb * slices) / a.ipc;
+                a.parts[(gb * a.max_parts + (blockIdx.x - first_cta)) * kTmaRows + lane] = tot;
+            } else {
+                const int64_t n = gb * kTmaRows + lane;
+                if (n < a.N) {
+                    if (XMODE == 1)
+                        a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f));
+                    else
+                        a.y_i32[n] = tot;
+                }
             }
         }
         acc[0] = acc[1] = acc[2] = acc[3] = 0;
         ncontrib = 0;
+        corr = 0;
     };
 
     // consume cursor
-    int64_t cbl = it_begin / slices;
-    int cj = (int)(it_begin - cbl * slices);
+    int cslot = (int)(p0 / slices), cj = (int)(p0 - (int64_t)(p0 / slices) * slices);
     for (int n = 0; n < n_items; ++n) {
         const int s = n % NS;
         if (!mbar_wait_bounded(&mybar[s], (uint32_t)(n / NS) & 1u)) {
@@ -298,13 +346,33 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
             mac_word(acc, w.w, x3);
         }
         ++ncontrib;
+        corr += qslice[cj];
         __syncwarp();
         if (lane == 0 && n + NS < n_items) issue_next(s);
         if (++cj == slices || n + 1 == n_items) {
-            flush(cbl);
+            flush(cslot);
             cj = 0;
-            ++cbl;
+            ++cslot;
         }
+    }
+}
+
+// Split-mode fixup: y[n] = sum of the int32 parts of n's row block, in CTA
+// order, then the int32 or BitLinear epilogue.
+__global__ void __launch_bounds__(256) gemv_tma_fixup_kernel(const GemvTmaArgs a) {
+    pdl_wait();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    float f = 0.0f;
+    if (a.y_bf16 != nullptr) f = __fdiv_rn(*a.gamma, *a.s_out);
+    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < a.N; n += stride) {
+        const int64_t b = n / kTmaRows;
+        const int64_t c0 = (b * a.slices) / a.ipc, c1 = ((b + 1) * a.slices - 1) / a.ipc;
+        int t = 0;
+        for (int64_t c = c0; c <= c1; ++c) t += a.parts[(b * a.max_parts + (c - c0)) * kTmaRows + (n % kTmaRows)];
+        if (a.y_bf16 != nullptr)
+            a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)t, f));
+        else
+            a.y_i32[n] = t;
     }
 }
 

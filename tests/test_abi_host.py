@@ -62,6 +62,15 @@ def test_workspace_bytes(lib):
     assert lib.bitnet_workspace_bytes(3, 100, 1000) == lib.bitnet_workspace_bytes(3, 100, 1000)
 
 
+# The tests below pass fake pointers; each call is built to fail a host-side
+# check before any device work.  They are skipped where a GPU is present, so
+# that a wrong expectation can never turn into a launch on fake pointers.
+def _no_gpu():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer host checks run only where no GPU is present")
+
+
 A = ctypes.c_void_p(0x10000)       # aligned fake device pointer
 A2 = ctypes.c_void_p(0x20000)
 MIS = ctypes.c_void_p(0x10001)     # misaligned
@@ -70,6 +79,7 @@ S = None                           # default stream
 
 
 def test_gemm_argument_errors(lib):
+    _no_gpu()
     g = lib.bitnet_w2a8_gemm
     assert g(A, A, A, -1, 4, 4, NULL, 0, S) == bn.BITNET_ERR_INVALID_ARG
     assert g(A, A, A, 1, 4, (1 << 21) + 1, NULL, 0, S) == bn.BITNET_ERR_INVALID_ARG
@@ -81,26 +91,31 @@ def test_gemm_argument_errors(lib):
     # empty problems are no-ops that touch nothing
     assert g(NULL, NULL, NULL, 0, 4, 4, NULL, 0, S) == bn.BITNET_OK
     assert g(NULL, NULL, NULL, 3, 0, 4, NULL, 0, S) == bn.BITNET_OK
-    # a split-K shape without enough workspace
-    need = lib.bitnet_workspace_bytes(1, 64, 65536)
-    assert need > 0
-    assert g(A, A, A, 1, 64, 65536, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
-    assert g(A, A, A, 1, 64, 65536, MIS, need, S) == bn.BITNET_ERR_ALIGNMENT
+    # K not a multiple of 16 with M >= 2: the activations are always repacked
+    # into the workspace, so one is required
+    need = lib.bitnet_workspace_bytes(2, 64, 1000)
+    assert need >= 2 * 1024
+    assert g(A, A, A, 2, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
+    assert g(A, A, A, 2, 64, 1000, A2, 64, S) == bn.BITNET_ERR_WORKSPACE
+    assert g(A, A, A, 2, 64, 1000, MIS, need, S) == bn.BITNET_ERR_ALIGNMENT
 
 
 def test_bitlinear_argument_errors(lib):
-    # every call here fails its host-side checks: none may reach a launch
+    # every call here fails its host-side checks: none may reach a launch.
+    # M >= 2: the quantised activations always go to the workspace
+    _no_gpu()
     f = lib.bitnet_bitlinear
-    ws_need = lib.bitnet_workspace_bytes(1, 64, 65536)  # a split-K shape: needs workspace
-    assert f(A, A, NULL, A, 1, 64, 65536, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
-    assert f(MIS, A, A, A, 1, 64, 65536, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
-    assert f(A, A, A, A, 1, 64, 65536, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 1, 64, 65536, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 1, 64, 65536, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    ws_need = lib.bitnet_workspace_bytes(2, 64, 1000)
+    assert f(A, A, NULL, A, 2, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
+    assert f(MIS, A, A, A, 2, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    assert f(A, A, A, A, 2, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 2, 64, 1000, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 2, 64, 1000, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
     assert f(NULL, NULL, NULL, NULL, 0, 8, 64, NULL, 0, S) == bn.BITNET_OK
 
 
 def test_prep_argument_errors(lib):
+    _no_gpu()
     assert lib.bitnet_absmean(A, 4, 4, NULL, A2, 8192, S) == bn.BITNET_ERR_INVALID_ARG
     assert lib.bitnet_absmean(A, 4, 4, A, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
     assert lib.bitnet_absmean(A, 4, 4, A, A2, 4, S) == bn.BITNET_ERR_WORKSPACE

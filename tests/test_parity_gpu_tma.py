@@ -1,7 +1,8 @@
 """Parity of the TMA-staged decode GEMV on small and ragged shapes.
 
 Full-size shapes reach the TMA path on their own (packed weights >= 6 MB); here
-a child process forces it (BITNET_GEMV_TUNE, read once per process) for shapes
+a child process forces it (BITNET_GEMV_TUNE, read once per process: whole row
+blocks per CTA or split mode, several warp/stage variants) for shapes
 with ragged row blocks (N not a multiple of 32), partial K-slices (K_pad/4 not
 a multiple of 128) and a single row block, int32 and fused-BitLinear outputs.
 """
@@ -46,12 +47,16 @@ print(json.dumps(out))
 """
 
 
-def test_tma_path_forced_small_shapes():
+@pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,1",    # TMA path, whole row blocks per CTA
+                                  "0,0,0,0,-1,1,1",    # TMA path, split mode (parts + fixup)
+                                  "0,0,0,0,-1,1,4",    # split mode, 8 warps x 2 boxes
+                                  "0,0,0,0,-1,0,5"])   # 4 warps x 4 boxes
+def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     env = dict(os.environ)
-    env["BITNET_GEMV_TUNE"] = "0,0,0,0,-1,0,1"  # TMA path whenever it applies
+    env["BITNET_GEMV_TUNE"] = tune
     code = "ROOT = " + repr(ROOT) + "\n" + CHILD
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]

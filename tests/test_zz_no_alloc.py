@@ -18,10 +18,16 @@ from ternary_weight_bit_w2a8_b200 import synth
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # checked on the host before any device work: fake pointers are never used
+    # checked on the host before any device work; the fake pointers are never
+    # used, and the test is skipped where a GPU is present so a wrong
+    # expectation cannot become a launch on them.  K not a multiple of 16 with
+    # M >= 2: the activations are repacked into M * K_pad bytes of scratch
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer host check runs only where no GPU is present")
     lib = bn.lib()
     A = ctypes.c_void_p(0x10000)
-    M, N, K = 4, 65536, 131072
+    M, N, K = 4, 64, (1 << 21) - 1
     assert lib.bitnet_workspace_bytes(M, N, K) > 1048576
     assert lib.bitnet_w2a8_gemm_noalloc(A, A, A, M, N, K, None) == bn.BITNET_ERR_WORKSPACE
     assert lib.bitnet_w2a8_gemm_noalloc(A, A, A, 0, N, K, None) == bn.BITNET_OK
