@@ -300,7 +300,9 @@ def measure_bitlinear_decode(torch, bn, shapes, warmup, l2_bytes, reps=30):
     return out
 
 
-def measure_prefill(torch, bn, ms_list, shapes, steps, warmup, int8_peak_tops):
+def measure_prefill(torch, bn, ms_list, shapes, warmup, int8_peak_tops, reps=20, L=10):
+    """Prefill GEMM (tcgen05, int32 out): mean per-call time in a graph of L
+    back-to-back calls; int8 TOPS = 2*M*N*K / time."""
     out = []
     for (N, K) in shapes:
         W = synth.bf16_weights(N, K, seed=1)
@@ -314,15 +316,44 @@ def measure_prefill(torch, bn, ms_list, shapes, steps, warmup, int8_peak_tops):
             q, s, _ = bn.bitnet_quant_act(xd)
             y = torch.empty((M, N), dtype=torch.int32, device="cuda")
             ws = bn.workspace(M, N, K)
-            g = capture(torch, lambda: bn.bitnet_w2a8_gemm(q, packed, N, y=y, ws=ws))
-            n = max(3, steps)
-            ms = timed_graph_loop(torch, [g], n, warmup)
-            us = ms * 1e3 / n
+
+            def run():
+                for _ in range(L):
+                    bn.bitnet_w2a8_gemm(q, packed, N, y=y, ws=ws)
+            g = capture(torch, run)
+            ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+            us = ms * 1e3 / (reps * L)
             tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
             out.append({"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "int8_TOPS": round(tops, 1),
                         "frac_int8_peak": round(tops / int8_peak_tops, 4),
                         "GBps": round(gemv_bytes(M, N, K) / (us * 1e-6) / 1e9, 1)})
             del g
+    return out
+
+
+def measure_bf16_context(torch, shapes, warmup, l2_bytes, reps=30):
+    """Context only (the pages compare their kernel with torch.matmul in bf16):
+    cuBLAS bf16 GEMV [1, K] x [K, N] for the sweep shapes, weights rotating as
+    for the W2A8 calls, mean per-call time in a graph of back-to-back calls."""
+    out = []
+    for (N, K) in shapes:
+        w = torch.randn((K, N), device="cuda", dtype=torch.bfloat16)
+        C = rotation_copies(w.numel() * 2, l2_bytes)
+        ws = [w] + [w.clone() for _ in range(C - 1)]
+        x = torch.randn((1, K), device="cuda", dtype=torch.bfloat16)
+        y = torch.empty((1, N), device="cuda", dtype=torch.bfloat16)
+        L = 4 * C
+
+        def run():
+            for i in range(L):
+                torch.matmul(x, ws[i % C], out=y)
+        g = capture(torch, run)
+        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+        us = ms * 1e3 / (reps * L)
+        out.append({"N": N, "K": K, "bf16_us_per_call": round(us, 3),
+                    "GBps": round((2 * N * K + 2 * K + 2 * N) / (us * 1e-6) / 1e9, 1)})
+        del g, ws
+        torch.cuda.empty_cache()
     return out
 
 
@@ -375,8 +406,12 @@ def run_ours(args, rank, world, dist):
         torch.cuda.empty_cache()
         details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
                                                                args.warmup, l2)
-        details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES,
-                                             max(10, min(args.steps // 20, 200)), max(3, args.warmup), int8_peak)
+        details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES, args.warmup, int8_peak)
+        bf = measure_bf16_context(torch, synth.SWEEP_SHAPES, args.warmup, l2)
+        for row, ours in zip(bf, details["sweep"]):
+            row["w2a8_us_per_call"] = ours["us_per_call"]
+            row["speedup_w2a8_vs_bf16"] = round(row["bf16_us_per_call"] / ours["us_per_call"], 2)
+        details["bf16_matmul_context"] = bf
         details["int8_peak_tops"] = {"value": round(int8_peak, 1),
                                      "basis": f"{peaks['source']} bf16 dense x 2 (nominal int8/bf16 ratio)"}
 
