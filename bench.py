@@ -133,6 +133,20 @@ def bf16_dev(torch, bits):
     return to_dev(torch, bits.view(np.int16)).view(torch.bfloat16)
 
 
+def max_over_ranks(torch, x, dist, device):
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbps(bytes_per_step_per_rank, steps, ms_max, world):
+    """Whole-job throughput: the bytes all ranks processed over the slowest rank's time."""
+    return world * bytes_per_step_per_rank * steps / (ms_max * 1e-3) / 1e9
+
+
 def timed_graph_loop(torch, graphs, steps, warmup, dist=None):
     """Replays graphs round-robin: `warmup` untimed, then exactly `steps` timed.
     Returns the elapsed ms (max over ranks)."""
@@ -149,11 +163,8 @@ def timed_graph_loop(torch, graphs, steps, warmup, dist=None):
         graphs[i % len(graphs)].replay()
     end.record()
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
+    ms = max_over_ranks(torch, start.elapsed_time(end), dist, "cuda")
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
 
@@ -377,17 +388,14 @@ def run_ours(args, rank, world, dist):
     ms, launches_per_step, clk = measure_gemv_set(torch, bn, gs, args.steps, args.warmup, dist, clocks)
     per_shape_us = per_launch_us(torch, bn, gs, args.warmup)
     ms_per_step = ms / args.steps
-    value = world * gs.bytes_per_step * args.steps / (ms * 1e-3) / 1e9
+    value = job_gbps(gs.bytes_per_step, args.steps, ms, world)
     kern_us = sum(per_shape_us)
     achieved = gs.bytes_per_step / (kern_us * 1e-6) / 1e9
 
     e2e_steps = max(3, min(args.steps, 300))
     e2e_ms, h2d, d2h = e2e_sweep(torch, bn, gs, e2e_steps)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * gs.bytes_per_step * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(torch, e2e_ms, dist, "cuda")
+    e2e_value = job_gbps(gs.bytes_per_step, e2e_steps, e2e_ms, world)
 
     details = {"sweep": [{"N": N, "K": K, "us_per_call": round(u, 3),
                           "GBps": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9, 1),
@@ -499,7 +507,7 @@ def run_reference(args):
     t0 = time.perf_counter()
     oracle_sweep_step(data, 1.0 / 64, 0)
     t_probe = (time.perf_counter() - t0) * 64  # seconds for one full sweep
-    budget = 90.0 / max(1, args.steps + args.warmup)  # whole run within ~1.5 min
+    budget = args.ref_budget / max(1, args.steps + args.warmup)  # whole run within the budget
     frac = min(1.0, budget / max(t_probe, 1e-9))
     for i in range(args.warmup):
         oracle_sweep_step(data, frac, i)
@@ -552,6 +560,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline only (skip the details workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--profile", metavar="M,N,K",
                     help="profiling mode: only `steps` plain bitnet_w2a8_gemm calls on one problem (for ncu)")
     args = ap.parse_args()
