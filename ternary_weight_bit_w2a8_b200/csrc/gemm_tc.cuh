@@ -10,7 +10,8 @@
 //   - CTA tile: 128 tokens (UMMA M) x BN weight rows (UMMA N) x 128 k per stage.
 //   - Warp 0, one lane: TMA producer.  Per stage it loads the activation tile
 //     (int8 [128 x 128 bytes], 128-byte swizzle: the canonical K-major operand
-//     layout) and the packed weight tile (layout v1, [BN rows x 32 bytes]).
+//     layout) into a ring of SAB stages and the packed weight tile (layout v1,
+//     [BN rows x 32 bytes], 32-byte swizzle) into a ring of SP stages.
 //   - Warps 2..5: decoders.  Each 32-bit packed word (16 consecutive k of one
 //     row) becomes 16 code bytes ((word >> 2j) & 0x03030303, j = 0..3), stored
 //     as the row's 16-byte chunk in the same swizzled K-major layout; then a
@@ -46,7 +47,6 @@ namespace bitnet {
 
 constexpr int kTcBM = 128;              // tokens per tile (UMMA M)
 constexpr int kTcBK = 128;              // k per stage (bytes of an activation row)
-constexpr int kTcStages = 3;
 constexpr int kTcThreads = 192;         // 6 warps
 constexpr int kTcAStageBytes = kTcBM * kTcBK;  // 16 KB
 constexpr int kTcOnesRows = 16;
@@ -63,16 +63,18 @@ struct GemmTcArgs {
     const float *gamma;     // weight scale (BitLinear)
 };
 
-template <int BN>
+// Shared-memory plan: SAB stages of (activation tile, decoded code tile), SP
+// stages of packed tiles (consumed by the decoders as soon as they land).
+template <int BN, int SAB, int SP>
 struct TcSmem {
     static constexpr int kBStage = BN * kTcBK;      // decoded codes
     static constexpr int kPStage = BN * 32;         // packed bytes
     static constexpr int kA = 0;
-    static constexpr int kB = kA + kTcStages * kTcAStageBytes;
-    static constexpr int kP = kB + kTcStages * kBStage;
-    static constexpr int kOnes = kP + kTcStages * kPStage;   // 1024-aligned: all the above are multiples of 1 KB
+    static constexpr int kB = kA + SAB * kTcAStageBytes;
+    static constexpr int kP = kB + SAB * kBStage;
+    static constexpr int kOnes = kP + SP * kPStage;   // 1024-aligned: all the above are multiples of 1 KB
     static constexpr int kBars = kOnes + kTcOnesRows * kTcBK;
-    static constexpr int kBarCount = 3 * kTcStages + 2;      // tma_full, dec_full, mma_done, accum_full, drain
+    static constexpr int kBarCount = 3 * SAB + 2 * SP + 2;  // a_full, dec_full, mma_done, p_full, p_empty, accum, drain
     static constexpr int kMisc = kBars + kBarCount * 8;      // tmem base (4 B) + abort flag (4 B)
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kTmemCols = (BN + kTcOnesRows) <= 128 ? 128 : ((BN + kTcOnesRows) <= 256 ? 256 : 512);
@@ -167,18 +169,20 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x,
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-template <int BN, bool BF16_OUT>
+template <int BN, bool BF16_OUT, int SAB, int SP>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
                         const __grid_constant__ CUtensorMap ymap, const GemmTcArgs a) {
-    using L = TcSmem<BN>;
+    using L = TcSmem<BN, SAB, SP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBars);
-    uint64_t *tma_full = bars;
-    uint64_t *dec_full = bars + kTcStages;
-    uint64_t *mma_done = bars + 2 * kTcStages;
-    uint64_t *accum_full = bars + 3 * kTcStages;
+    uint64_t *a_full = bars;
+    uint64_t *dec_full = bars + SAB;
+    uint64_t *mma_done = bars + 2 * SAB;
+    uint64_t *p_full = bars + 3 * SAB;
+    uint64_t *p_empty = p_full + SP;
+    uint64_t *accum_full = p_empty + SP;
     uint64_t *drain = accum_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kMisc + 4);
@@ -190,10 +194,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     // ---- set-up: barriers, the ones tile, tensor memory
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(&tma_full[s], 1);
+        for (int s = 0; s < SAB; ++s) {
+            mbar_init(&a_full[s], 1);
             mbar_init(&dec_full[s], 4);   // one arrival per decoder warp
             mbar_init(&mma_done[s], 1);
+        }
+        for (int s = 0; s < SP; ++s) {
+            mbar_init(&p_full[s], 1);
+            mbar_init(&p_empty[s], 4);    // one arrival per decoder warp
         }
         mbar_init(accum_full, 1);
         mbar_init(drain, 1);
@@ -219,21 +227,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        int issued = 0;
         if (lane == 0) {
             pdl_wait();
+            int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kTcStages;
-                if (kb >= kTcStages && !tc_wait(&mma_done[s], (uint32_t)((kb / kTcStages) - 1) & 1u, abort_flag))
-                    break;
-                mbar_arrive_expect_tx(&tma_full[s], kTcAStageBytes + L::kPStage);
-                tma_load_2d(sm + L::kA + s * kTcAStageBytes, &amap, (kbase + kb) * kTcBK, (int)m0, &tma_full[s]);
-                tma_load_2d(sm + L::kP + s * L::kPStage, &pmap, (kbase + kb) * 32, (int)n0, &tma_full[s]);
+                const int s = kb % SAB, ps = kb % SP;
+                if (kb >= SAB && !tc_wait(&mma_done[s], (uint32_t)((kb / SAB) - 1) & 1u, abort_flag)) break;
+                if (kb >= SP && !tc_wait(&p_empty[ps], (uint32_t)((kb / SP) - 1) & 1u, abort_flag)) break;
+                mbar_arrive_expect_tx(&a_full[s], kTcAStageBytes);
+                tma_load_2d(sm + L::kA + s * kTcAStageBytes, &amap, (kbase + kb) * kTcBK, (int)m0, &a_full[s]);
+                mbar_arrive_expect_tx(&p_full[ps], L::kPStage);
+                tma_load_2d(sm + L::kP + ps * L::kPStage, &pmap, (kbase + kb) * 32, (int)n0, &p_full[ps]);
                 issued = kb + 1;
             }
             // make sure no copy is still landing in shared memory when the CTA leaves
-            for (int kb = issued - kTcStages < 0 ? 0 : issued - kTcStages; kb < issued; ++kb)
-                mbar_wait_bounded(&tma_full[kb % kTcStages], (uint32_t)(kb / kTcStages) & 1u);
+            for (int kb = issued - SAB < 0 ? 0 : issued - SAB; kb < issued; ++kb)
+                mbar_wait_bounded(&a_full[kb % SAB], (uint32_t)(kb / SAB) & 1u);
+            for (int kb = issued - SP < 0 ? 0 : issued - SP; kb < issued; ++kb)
+                mbar_wait_bounded(&p_full[kb % SP], (uint32_t)(kb / SP) & 1u);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
@@ -243,8 +254,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t ones = smem_u32(sm + L::kOnes);
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kTcStages;
-                if (!tc_wait(&dec_full[s], (uint32_t)(kb / kTcStages) & 1u, abort_flag)) {
+                const int s = kb % SAB;
+                if (!tc_wait(&dec_full[s], (uint32_t)(kb / SAB) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -273,12 +284,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int t = threadIdx.x - 64;  // 0..127
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kTcStages;
-            if (!tc_wait(&tma_full[s], (uint32_t)(kb / kTcStages) & 1u, abort_flag)) {
+            const int s = kb % SAB, pst = kb % SP;
+            // the packed tile has landed; the activation tile of this stage has too,
+            // which also means the MMAs that last read this stage's code tile are done
+            if (!tc_wait(&p_full[pst], (uint32_t)(kb / SP) & 1u, abort_flag) ||
+                !tc_wait(&a_full[s], (uint32_t)(kb / SAB) & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
-            const uint8_t *ps = sm + L::kP + s * L::kPStage;
+            const uint8_t *ps = sm + L::kP + pst * L::kPStage;
             uint8_t *bs = sm + L::kB + s * L::kBStage;
 #pragma unroll
             for (int n = t; n < BN; n += 128) {
@@ -298,7 +312,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // codes -> tensor core
             __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&dec_full[s])) : "memory");
+            if (lane == 0) {
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&p_empty[pst])) : "memory");
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&dec_full[s])) : "memory");
+            }
         }
         // epilogue: thread t owns accumulator row (warp % 4) * 32 + lane
         if (ok && tc_wait(accum_full, 0, abort_flag)) {
