@@ -36,7 +36,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[10] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    size_t tma_max_dyn[22] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[8] = {false, false, false, false, false, false, false, false};
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -208,21 +208,34 @@ constexpr int kTmaNumCfg = 5;
 constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
-TmaKernel tma_kernel_for(int xmode, int cfg) {
-    static const TmaKernel table[2 * kTmaNumCfg] = {
-        gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 12, 3>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 2>,
-        gemv_tma_kernel<0, 4, 4>, gemv_tma_kernel<1, 8, 4>,  gemv_tma_kernel<1, 12, 3>, gemv_tma_kernel<1, 16, 2>,
-        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 4, 4>};
-    return table[xmode * kTmaNumCfg + cfg];
+// Kernel of (mode, variant, tokens per launch).  Several tokens (MT = 2, 4, 8)
+// are compiled for the 8 x 4 and 16 x 2 variants only; slot in the
+// shared-memory opt-in table: xmode * 11 + (MT == 1 ? cfg : 5 + 2 * log2(MT / 2) + (cfg == 2)).
+int tma_kernel_slot(int xmode, int cfg, int mt) {
+    const int base = mt == 1 ? cfg : 5 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (cfg == 2 ? 1 : 0);
+    return xmode * 11 + base;
+}
+
+TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
+    static const TmaKernel table[22] = {
+        gemv_tma_kernel<0, 8, 4, 1>, gemv_tma_kernel<0, 12, 3, 1>, gemv_tma_kernel<0, 16, 2, 1>,
+        gemv_tma_kernel<0, 8, 2, 1>, gemv_tma_kernel<0, 4, 4, 1>,
+        gemv_tma_kernel<0, 8, 4, 2>, gemv_tma_kernel<0, 16, 2, 2>, gemv_tma_kernel<0, 8, 4, 4>,
+        gemv_tma_kernel<0, 16, 2, 4>, gemv_tma_kernel<0, 8, 4, 8>, gemv_tma_kernel<0, 16, 2, 8>,
+        gemv_tma_kernel<1, 8, 4, 1>, gemv_tma_kernel<1, 12, 3, 1>, gemv_tma_kernel<1, 16, 2, 1>,
+        gemv_tma_kernel<1, 8, 2, 1>, gemv_tma_kernel<1, 4, 4, 1>,
+        gemv_tma_kernel<1, 8, 4, 2>, gemv_tma_kernel<1, 16, 2, 2>, gemv_tma_kernel<1, 8, 4, 4>,
+        gemv_tma_kernel<1, 16, 2, 4>, gemv_tma_kernel<1, 8, 4, 8>, gemv_tma_kernel<1, 16, 2, 8>};
+    return table[tma_kernel_slot(xmode, cfg, mt)];
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    size_t &slot = dev->tma_max_dyn[xmode * kTmaNumCfg + cfg];
+    size_t &slot = dev->tma_max_dyn[tma_kernel_slot(xmode, cfg, mt)];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, cfg);
+        TmaKernel kern = tma_kernel_for(xmode, cfg, mt);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -238,6 +251,7 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg) {
 struct TmaPlan {
     bool use;
     int cfg, slices, max_blocks, grid, max_parts;
+    int mt;            // tokens per launch (1, 2, 4, 8)
     int64_t ipc;       // > 0: split mode
     size_t smem;
     int64_t ws_bytes;  // split mode: int32 parts and the BitLinear scale
@@ -248,7 +262,8 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     constexpr size_t kRefSmemPerSM = 233472, kRefCtaReserve = 1024, kRefSmemOptin = 232448;
     TmaPlan p{};
     const int tune = gemv_tune().tma;
-    if (M != 1 || tune == 0 || K < kTmaSliceK || N < 1) return p;
+    if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
+    p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
     const int64_t row_bytes = packed_row_bytes(K);
     const int64_t nblocks = ceil_div(N, kTmaRows);
     p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
@@ -258,9 +273,10 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
         p.cfg = tune - 1;
     else
         p.cfg = N * row_bytes < (3ll << 20) ? 0 : (p.slices >= 32 ? 1 : 2);
+    if (p.mt > 1 && p.cfg != 0) p.cfg = 2;  // several tokens: 8 x 4 or 16 x 2 only
     const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
     // resident CTAs per SM for the block-strided layout (accumulator slots are small)
-    const size_t base_smem = gemv_tma_smem_bytes(W, NS, p.slices, 1);
+    const size_t base_smem = gemv_tma_smem_bytes(W, NS, p.slices, 1, p.mt);
     int per_sm = (int)(kRefSmemPerSM / (base_smem + kRefCtaReserve));
     if (per_sm > 2048 / (W * 32)) per_sm = 2048 / (W * 32);
     if (per_sm < 1) return p;
@@ -274,7 +290,7 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     // every shape tried, so split mode is used only when asked for)
     (void)mean;
     (void)worst;
-    const bool want_split = gemv_tune().S == 1;
+    const bool want_split = gemv_tune().S == 1 && p.mt == 1;
     if (want_split) {
         const int64_t items = nblocks * p.slices;
         p.ipc = ceil_div(items, gmax);
@@ -286,16 +302,17 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
         p.grid = (int)g_strided;
         p.max_blocks = (int)ceil_div(nblocks, g_strided);
     }
-    p.smem = gemv_tma_smem_bytes(W, NS, p.slices, p.max_blocks);
+    p.smem = gemv_tma_smem_bytes(W, NS, p.slices, p.max_blocks, p.mt);
     if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
     p.use = true;
     return p;
 }
 
-int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t N,
-                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const TmaPlan &tp, void *ws,
-                    cudaStream_t st) {
-    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg)) return BITNET_ERR_CUDA;
+int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
+                    int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
+                    const TmaPlan &tp, void *ws, cudaStream_t st) {
+    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt))
+        return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
     const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
@@ -306,7 +323,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
                              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return BITNET_ERR_CUDA;
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg);
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
     // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
     // makes one wait run out, exercising the device-timeout path
     static std::atomic<int> stall_once{-1};
@@ -320,6 +337,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     GemvTmaArgs a{};
     a.q = q;
     a.x = x;
+    a.M = (int)M;
     a.N = N;
     a.K = K;
     a.slices = tp.slices;
@@ -329,6 +347,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
+    a.s_act = s_act;
     a.test_stall = test_stall;
     a.ipc = tp.ipc;
     a.max_parts = tp.max_parts;
@@ -348,7 +367,8 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
                 const float *s_act, const float *gamma, void *ws, cudaStream_t st) {
     {
         const TmaPlan tp = tma_plan(M, N, K);
-        if (tp.use) return launch_gemv_tma(dev, xmode, q, x, packed, N, K, y_i32, y_bf16, gamma, tp, ws, st);
+        if (tp.use && ldq == K)
+            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, ws, st);
     }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();
@@ -608,6 +628,17 @@ struct GemmPlan {
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinear) {
     GemmPlan p{};
+    (void)q_tma_ok;
+    if (M <= 8) {  // decode and small batches: the TMA GEMV reads the weights once
+        const TmaPlan tp = tma_plan(M, N, K);
+        if (tp.use) {
+            p.path = kPathGemv;
+            p.ws_bytes = tp.ws_bytes;
+            // BitLinear on several tokens quantises them once into the workspace
+            if (bitlinear && M >= 2) p.ws_bytes = round_up(M * K, 256) + round_up(M * 4, 256);
+            return p;
+        }
+    }
     if (M >= 2 && K >= kTcBK) {
         p.path = kPathTc;
         p.tc = tc_plan(M, N, K);
@@ -791,6 +822,14 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     if (K == 0) {
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
+    }
+    if (p.path == kPathGemv && M >= 2 && M <= 8 && tma_plan(M, N, K).use) {
+        // small batch: quantise the tokens once, then one pass over the weights
+        int8_t *q = static_cast<int8_t *>(workspace);
+        float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * K, 256));
+        quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, K, false, s, nullptr);
+        if ((rc = launched()) != BITNET_OK) return rc;
+        return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, nullptr, y, s, gamma, nullptr, st);
     }
     if (p.path == kPathGemv)  // activations quantised per token inside the GEMV: one launch
         return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);

@@ -1,5 +1,5 @@
-// gemv_tma.cuh -- the decode GEMV for large weight matrices: packed weights
-// stream through shared memory by TMA, one row per lane.
+// gemv_tma.cuh -- the decode GEMV (one to eight tokens): packed weights stream
+// through shared memory by TMA, one row per lane.
 //
 // Same contraction and decode as gemv.cuh (layout v1 words, shift-free dp4a
 // on codes scaled by 4^j, activation-sum correction); what differs is how the
@@ -16,8 +16,10 @@
 //     lane 0 issues the TMA for the item NS ahead as soon as the warp has read
 //     a stage, so up to NS boxes per warp are in flight without holding
 //     registers.
-//   - Activations live in shared memory as one linear array; all lanes read
-//     the same 16 bytes at a time (a broadcast).
+//   - Activations live in shared memory as one linear array per token; all
+//     lanes read the same 16 bytes at a time (a broadcast).  With several
+//     tokens (MT = 2, 4, 8) every weight box is still read from HBM once: the
+//     four code masks of each word are computed once and reused per token.
 //   - A warp adds its per-row partial sums into a per-row-block int32
 //     accumulator in shared memory (atomics: exact and order-free) whenever its
 //     item sequence leaves a row block; the warp whose contribution completes
@@ -46,6 +48,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s per wait
 struct GemvTmaArgs {
     const int8_t *q;      // int8 activations [M, K] (mode 0)
     const uint16_t *x;    // bf16 activations [M, K] (mode 1)
+    int M;                // tokens of this launch (<= the kernel's MT)
     int64_t N, K;
     int slices;           // K-slices of 128 packed bytes per row
     int64_t blk_begin;    // first row block of this launch
@@ -61,15 +64,17 @@ struct GemvTmaArgs {
     int32_t *y_i32;       // [M, N] int32 result
     uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
     const float *gamma;   // weight scale (BitLinear)
+    const float *s_act;   // mode 0 with bf16 output: per-token activation scales [M]
     int test_stall;       // test hook: warp 0 never requests its first box, so its first wait times out
 };
 
 // Dynamic shared memory of a launch: ring of warps x stages boxes, linear
 // activations, per-row-block accumulators and counters, mbarriers.
-__host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta) {
-    return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes + (size_t)slices * kTmaSliceK +
-           (size_t)max_blocks_cta * kTmaRows * 4 + (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 +
-           (size_t)slices * 4;
+__host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta,
+                                                      int tokens = 1) {
+    return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes +
+           (size_t)tokens * slices * kTmaSliceK + (size_t)max_blocks_cta * tokens * kTmaRows * 4 +
+           (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -195,24 +200,26 @@ __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, floa
     return sc;
 }
 
-template <int XMODE, int W, int NS>
+template <int XMODE, int W, int NS, int MT>
 __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
+    static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8, "tokens per launch");
     extern __shared__ uint8_t smem_raw[];
     __shared__ float red[32];
     // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8 rows
     // of 128 bytes); computed on the shared-window address so that every
     // pointer below stays a shared-memory pointer
     uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * NS * kTmaBoxBytes);
+    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * NS * kTmaBoxBytes);   // [MT][kq]
     const int64_t kq = (int64_t)a.slices * kTmaSliceK;
-    int *accs = reinterpret_cast<int *>(qlin + kq);
-    int *done = accs + a.max_blocks_cta * kTmaRows;
-    int *qslice = done + a.max_blocks_cta;   // activation sum of each K-slice
-    uint64_t *bars = reinterpret_cast<uint64_t *>(qslice + a.slices + ((a.max_blocks_cta + a.slices) & 1));
+    int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][32]
+    int *done = accs + a.max_blocks_cta * MT * kTmaRows;
+    int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
+    uint64_t *bars =
+        reinterpret_cast<uint64_t *>(qslice + MT * a.slices + ((a.max_blocks_cta + MT * a.slices) & 1));
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slices = a.slices;
-    const bool split = a.ipc > 0;
+    const bool split = a.ipc > 0;  // (single-token launches only)
     // this CTA's items, in (row block, slice) order; `bstep` is the distance
     // between consecutive row blocks of the CTA
     int64_t cta_begin, items, first_block, bstep;
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     uint8_t *myring = ring + warp * NS * kTmaBoxBytes;
 
     if (threadIdx.x < W * NS) mbar_init(&bars[threadIdx.x], 1);
-    for (int i = threadIdx.x; i < nslots * kTmaRows; i += blockDim.x) accs[i] = 0;
+    for (int i = threadIdx.x; i < nslots * MT * kTmaRows; i += blockDim.x) accs[i] = 0;
     for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
@@ -272,23 +279,45 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     pdl_launch_dependents();
     pdl_wait();
 
-    float sc = 0.0f;
-    if (XMODE == 0)
-        stage_qlin_int8(qlin, qslice, a.q, a.K, kq);
-    else
-        sc = stage_qlin_bf16(qlin, qslice, red, a.x, a.K, kq);
-    if (split && XMODE == 1 && a.s_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.s_out = sc;
+    float sc[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        sc[t] = 0.0f;
+        int8_t *qt = qlin + t * kq;
+        int *qst = qslice + t * slices;
+        if (t < a.M) {
+            if (XMODE == 0)
+                stage_qlin_int8(qt, qst, a.q + (int64_t)t * a.K, a.K, kq);
+            else
+                sc[t] = stage_qlin_bf16(qt, qst, red, a.x + (int64_t)t * a.K, a.K, kq);
+        } else {  // unused token slot: zeros, contributes nothing and is not stored
+            for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x)
+                reinterpret_cast<uint4 *>(qt)[p] = make_uint4(0u, 0u, 0u, 0u);
+            for (int j = threadIdx.x; j < slices; j += blockDim.x) qst[j] = 0;
+        }
+    }
+    if (split && XMODE == 1 && a.s_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.s_out = sc[0];
     __syncthreads();
-    float f = 0.0f;
-    if (XMODE == 1 && !split) f = __fdiv_rn(*a.gamma, sc);
+    float f[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        f[t] = 0.0f;
+        if (!split && t < a.M && a.y_bf16 != nullptr)
+            f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
+    }
 
-    int acc[4] = {0, 0, 0, 0};
-    int ncontrib = 0, corr = 0;
+    int acc[MT][4], corr[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
+    int ncontrib = 0;
     // folds this warp's partial sums of slot `sl` into shared memory; the warp
-    // completing the slot's items writes its 32 results (split mode: its part)
+    // completing the slot's items writes its results (split mode: its part)
     auto flush = [&](int sl) {
-        const int v = acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6) - corr;
-        atomicAdd(&accs[sl * kTmaRows + lane], v);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            const int v = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) - corr[t];
+            atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], v);
+        }
         __threadfence_block();
         __syncwarp();
         const int64_t blk = first_block + (int64_t)sl * bstep;
@@ -302,24 +331,25 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
         fin = __shfl_sync(0xffffffffu, fin, 0);
         if (fin) {
             __threadfence_block();
-            const int tot = atomicAdd(&accs[sl * kTmaRows + lane], 0);
             const int64_t gb = a.blk_begin + blk;
-            if (split) {
-                const int64_t first_cta = (gb * slices) / a.ipc;
-                a.parts[(gb * a.max_parts + (blockIdx.x - first_cta)) * kTmaRows + lane] = tot;
-            } else {
-                const int64_t n = gb * kTmaRows + lane;
-                if (n < a.N) {
-                    if (XMODE == 1)
-                        a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f));
+            const int64_t n = gb * kTmaRows + lane;
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                const int tot = atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], 0);
+                if (split) {
+                    const int64_t first_cta = (gb * slices) / a.ipc;
+                    a.parts[(gb * a.max_parts + (blockIdx.x - first_cta)) * kTmaRows + lane] = tot;
+                } else if (t < a.M && n < a.N) {
+                    if (a.y_bf16 != nullptr)
+                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
                     else
-                        a.y_i32[n] = tot;
+                        a.y_i32[(int64_t)t * a.N + n] = tot;
                 }
             }
         }
-        acc[0] = acc[1] = acc[2] = acc[3] = 0;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
         ncontrib = 0;
-        corr = 0;
     };
 
     // consume cursor
@@ -338,15 +368,41 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (lane & 7)) << 4));
-            const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
-            const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];
-            mac_word(acc, w.x, x0);
-            mac_word(acc, w.y, x1);
-            mac_word(acc, w.z, x2);
-            mac_word(acc, w.w, x3);
+            if (MT == 1) {
+                const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
+                const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];
+                mac_word(acc[0], w.x, x0);
+                mac_word(acc[0], w.y, x1);
+                mac_word(acc[0], w.z, x2);
+                mac_word(acc[0], w.w, x3);
+            } else {
+                // the four scaled code masks of each word, shared by all tokens
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                uint32_t mk[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    mk[i][0] = ww[i] & 0x03030303u;
+                    mk[i][1] = ww[i] & 0x0C0C0C0Cu;
+                    mk[i][2] = ww[i] & 0x30303030u;
+                    mk[i][3] = ww[i] & 0xC0C0C0C0u;
+                }
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const uint4 *qp = reinterpret_cast<const uint4 *>(qk + t * kq + c * 64);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 x = qp[i];
+                        acc[t][0] = dp4a_us(mk[i][0], x.x, acc[t][0]);
+                        acc[t][1] = dp4a_us(mk[i][1], x.y, acc[t][1]);
+                        acc[t][2] = dp4a_us(mk[i][2], x.z, acc[t][2]);
+                        acc[t][3] = dp4a_us(mk[i][3], x.w, acc[t][3]);
+                    }
+                }
+            }
         }
         ++ncontrib;
-        corr += qslice[cj];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) corr[t] += qslice[t * slices + cj];
         __syncwarp();
         if (lane == 0 && n + NS < n_items) issue_next(s);
         if (++cj == slices || n + 1 == n_items) {

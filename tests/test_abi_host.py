@@ -91,26 +91,26 @@ def test_gemm_argument_errors(lib):
     # empty problems are no-ops that touch nothing
     assert g(NULL, NULL, NULL, 0, 4, 4, NULL, 0, S) == bn.BITNET_OK
     assert g(NULL, NULL, NULL, 3, 0, 4, NULL, 0, S) == bn.BITNET_OK
-    # K not a multiple of 16 with M >= 2: the activations are always repacked
-    # into the workspace, so one is required
-    need = lib.bitnet_workspace_bytes(2, 64, 1000)
-    assert need >= 2 * 1024
-    assert g(A, A, A, 2, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
-    assert g(A, A, A, 2, 64, 1000, A2, 64, S) == bn.BITNET_ERR_WORKSPACE
-    assert g(A, A, A, 2, 64, 1000, MIS, need, S) == bn.BITNET_ERR_ALIGNMENT
+    # a prefill batch (tensor-core path) with K not a multiple of 16: the
+    # activations are always repacked into the workspace, so one is required
+    need = lib.bitnet_workspace_bytes(200, 64, 1000)
+    assert need >= 200 * 1024
+    assert g(A, A, A, 200, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
+    assert g(A, A, A, 200, 64, 1000, A2, 64, S) == bn.BITNET_ERR_WORKSPACE
+    assert g(A, A, A, 200, 64, 1000, MIS, need, S) == bn.BITNET_ERR_ALIGNMENT
 
 
 def test_bitlinear_argument_errors(lib):
     # every call here fails its host-side checks: none may reach a launch.
-    # M >= 2: the quantised activations always go to the workspace
+    # a prefill batch: the quantised activations always go to the workspace
     _no_gpu()
     f = lib.bitnet_bitlinear
-    ws_need = lib.bitnet_workspace_bytes(2, 64, 1000)
-    assert f(A, A, NULL, A, 2, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
-    assert f(MIS, A, A, A, 2, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
-    assert f(A, A, A, A, 2, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 2, 64, 1000, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
-    assert f(A, A, A, A, 2, 64, 1000, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    ws_need = lib.bitnet_workspace_bytes(200, 64, 1000)
+    assert f(A, A, NULL, A, 200, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_INVALID_ARG  # gamma
+    assert f(MIS, A, A, A, 200, 64, 1000, A2, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
+    assert f(A, A, A, A, 200, 64, 1000, NULL, 0, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 200, 64, 1000, A2, 16, S) == bn.BITNET_ERR_WORKSPACE
+    assert f(A, A, A, A, 200, 64, 1000, MIS, ws_need, S) == bn.BITNET_ERR_ALIGNMENT
     assert f(NULL, NULL, NULL, NULL, 0, 8, 64, NULL, 0, S) == bn.BITNET_OK
 
 

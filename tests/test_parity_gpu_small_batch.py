@@ -1,0 +1,48 @@
+"""Parity of the small-batch decode (2..8 tokens through the TMA-staged GEMV,
+every weight box read once for all tokens): int32 and BitLinear outputs on
+ragged shapes and token counts that leave unused token slots."""
+import numpy as np
+import pytest
+
+import oracle
+import ternary_weight_bit_w2a8_b200 as bn
+from ternary_weight_bit_w2a8_b200 import synth
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from ternary_weight_bit_w2a8_b200 import build
+    build.build()
+    yield
+    torch.cuda.synchronize()
+    assert bn.bitnet_get_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 1000, 2560), (3, 33, 700), (4, 257, 1024), (5, 300, 5120), (7, 64, 3200),
+                                   (8, 2560, 6912), (6, 13824, 2560)])
+def test_small_batch_int32_exact(M, N, K):
+    q, w = synth.uniform_int8_ternary(N, K, seed=M * 1000 + N + K, M=M)
+    q[-1, :7] = -128
+    y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
+    assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w))
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 500, 2560), (3, 6912, 2560), (8, 2560, 6912)])
+def test_small_batch_bitlinear(M, N, K):
+    x, W = synth.bitlinear_inputs(M, N, K, seed=M)
+    x[1] = 0  # a zero token among them
+    g = oracle.absmean(W)
+    wt = oracle.ternarize(W, g)
+    y = bn.bitnet_bitlinear(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16),
+                            bn.bitnet_pack_weights(torch.from_numpy(wt).cuda()),
+                            torch.tensor([float(g)], dtype=torch.float32, device="cuda"), N)
+    y_ref = oracle.bitlinear(x, wt, g)[0]
+    yf = y.float().cpu().numpy().astype(np.float64)
+    err = np.abs(yf - y_ref)
+    assert np.where(np.abs(y_ref) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(y_ref)).all()
+    assert not y.view(torch.int16).cpu().numpy()[1].any()
