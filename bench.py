@@ -147,11 +147,23 @@ def job_gbps(bytes_per_step_per_rank, steps, ms_max, world):
     return world * bytes_per_step_per_rank * steps / (ms_max * 1e-3) / 1e9
 
 
-def timed_graph_loop(torch, graphs, steps, warmup, dist=None):
-    """Replays graphs round-robin: `warmup` untimed, then exactly `steps` timed.
+def replay_steps(graphs, n, multi=None):
+    """Runs exactly `n` steps: `graphs[c]` is one step over rotation copy c;
+    `multi` (optional) holds all len(graphs) steps, copy 0 first, in one graph."""
+    C = len(graphs)
+    i = 0
+    if multi is not None:
+        for _ in range(n // C):
+            multi.replay()
+        i = (n // C) * C
+    for j in range(i, n):
+        graphs[j % C].replay()
+
+
+def timed_graph_loop(torch, graphs, steps, warmup, dist=None, multi=None):
+    """`warmup` untimed steps, then exactly `steps` timed ones (see replay_steps).
     Returns the elapsed ms (max over ranks)."""
-    for i in range(warmup):
-        graphs[i % len(graphs)].replay()
+    replay_steps(graphs, warmup, multi)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -159,8 +171,7 @@ def timed_graph_loop(torch, graphs, steps, warmup, dist=None):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record()
-    for i in range(steps):
-        graphs[i % len(graphs)].replay()
+    replay_steps(graphs, steps, multi)
     end.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(torch, start.elapsed_time(end), dist, "cuda")
@@ -221,17 +232,19 @@ class GemvSet:
 
 
 def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
-    """Headline: one graph per rotation copy holding one step (the calls of all
-    shapes back to back, linked by programmatic dependent launch), replayed
-    round-robin for exactly `steps` steps."""
+    """Headline: a step is the calls of all shapes back to back (linked by
+    programmatic dependent launch) over one rotation copy.  One graph holds the
+    steps of all copies in turn and is replayed whole; single-step graphs run
+    the remainder, so exactly `steps` steps are timed."""
     n_before = bn.bitnet_launch_count()
     graphs = [capture(torch, lambda c=c: gs.run(c)) for c in range(len(gs.copies))]
     launches_per_step = (bn.bitnet_launch_count() - n_before) // (2 * len(gs.copies))
+    multi = capture(torch, lambda: [gs.run(c) for c in range(len(gs.copies))])
     if clocks is not None:
         clocks.start()
-    ms = timed_graph_loop(torch, graphs, steps, warmup, dist)
+    ms = timed_graph_loop(torch, graphs, steps, warmup, dist, multi)
     clk = clocks.stop() if clocks is not None else None
-    del graphs
+    del graphs, multi
     return ms, launches_per_step, clk
 
 
@@ -424,6 +437,9 @@ def run_ours(args, rank, world, dist):
                                      "basis": f"{peaks['source']} bf16 dense x 2 (nominal int8/bf16 ratio)"}
 
     err = bn.bitnet_get_device_error()
+    traffic = read_traffic()
+    if traffic is not None:
+        traffic = round(traffic, 1)
     return {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -433,11 +449,15 @@ def run_ours(args, rank, world, dist):
                    "l2": f"weights rotate over {len(synth.SWEEP_SHAPES)}-shape sets, "
                          f"{rotation_copies(sum(N * K // 4 for N, K in synth.SWEEP_SHAPES), l2)} copies "
                          f"(> 2x L2 of {l2 // 2**20} MiB between reuses)",
-                   "step": "one CUDA-graph replay of the 8 bitnet_w2a8_gemm calls",
+                   "step": "the 8 bitnet_w2a8_gemm calls over one rotation copy; CUDA graphs of one step per "
+                           "copy, run as one graph of all copies in turn plus single steps for the remainder",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "seed": "rank"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "traffic_source": "profiles/traffic_gemv_tma_sweep.md (ncu dram__bytes_read.sum + "
+                                       "dram__bytes_write.sum, mean over the 8 sweep launches); null when the "
+                                       "kernel sources changed since that capture",
                      "kernel": "gemv_tma_kernel", "peak_source": peaks["source"],
                      "per_launch_bytes": "N*K/4 + K + 4N per shape, mean over the 8 shapes",
                      "duration": "mean per-call time of each shape in a graph of back-to-back calls over rotating "
@@ -529,10 +549,50 @@ def run_reference(args):
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "traffic_gemv_tma_sweep.md")
+TRAFFIC_SOURCES = ("common.cuh", "gemv_tma.cuh", "bitnet_b200.cu")
+
+
+def kernel_source_hash():
+    """sha256 over the sources that decide the GEMV kernel and its launch."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "ternary_weight_bit_w2a8_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def read_traffic(path=TRAFFIC_SUMMARY):
+    """DRAM bytes per launch (read + write, mean over the sweep's launches) from
+    the committed ncu summary, or None when the kernel sources changed since."""
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            key = line.split(":", 1)[0].strip()
+            if ":" in line and key in ("source_sha256", "traffic_bytes_per_launch"):
+                fields[key] = line.split(":", 1)[1].strip().strip("`")
+    if fields.get("source_sha256") != kernel_source_hash() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return float(fields["traffic_bytes_per_launch"])
+
+
 def run_profile(args):
-    """One problem, `steps` plain calls over rotating weight copies, no graphs."""
+    """`warmup + steps` plain calls over rotating weight copies, no graphs: of one
+    problem (M,N,K), or with `sweep` of each sweep shape at M = 1, in order."""
     import torch
     import ternary_weight_bit_w2a8_b200 as bn
+    if args.profile == "sweep":
+        l2 = torch.cuda.get_device_properties(0).L2_cache_size
+        gs = GemvSet(torch, bn, synth.SWEEP_SHAPES, synth.uniform_int8_ternary, seed=0, l2_bytes=l2)
+        for i in range(args.warmup + args.steps):
+            gs.run(i % len(gs.copies))
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": "sweep", "calls": (args.warmup + args.steps) * len(gs.shapes),
+                          "device_error": bn.bitnet_get_device_error()}))
+        return 0
     M, N, K = (int(v) for v in args.profile.split(","))
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     gen = synth.sparse_ternary_normal_int8 if (N, K) in synth.LARGE_SHAPES else synth.uniform_int8_ternary
@@ -562,8 +622,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work for the whole --impl reference run")
-    ap.add_argument("--profile", metavar="M,N,K",
-                    help="profiling mode: only `steps` plain bitnet_w2a8_gemm calls on one problem (for ncu)")
+    ap.add_argument("--profile", metavar="M,N,K|sweep",
+                    help="profiling mode: only plain bitnet_w2a8_gemm calls, `warmup + steps` of one problem "
+                         "or of each sweep shape (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -83,3 +83,32 @@ def test_reference_arm_other_ranks_exit_quietly():
                    {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_traffic_valid_only_for_the_captured_sources(tmp_path):
+    h = bench.kernel_source_hash()
+    good = tmp_path / "t.md"
+    good.write_text(f"notes: x\nsource_sha256: `{h}`\ntraffic_bytes_per_launch: `1234.5`\n")
+    assert bench.read_traffic(str(good)) == 1234.5
+    stale = tmp_path / "s.md"
+    stale.write_text("source_sha256: `" + "0" * 64 + "`\ntraffic_bytes_per_launch: `1234.5`\n")
+    assert bench.read_traffic(str(stale)) is None
+    assert bench.read_traffic(str(tmp_path / "missing.md")) is None
+
+
+def test_replay_steps_runs_exactly_n_steps():
+    class G:
+        def __init__(self, log, tag):
+            self.log, self.tag = log, tag
+
+        def replay(self):
+            self.log.append(self.tag)
+
+    for n in (0, 1, 6, 7, 15, 20):
+        log = []
+        singles = [G(log, (c,)) for c in range(7)]
+        multi = G(log, tuple(range(7)))
+        bench.replay_steps(singles, n, multi)
+        steps = [c for t in log for c in t]
+        assert len(steps) == n
+        assert steps == [i % 7 for i in range(n)]  # every step on the next rotation copy
