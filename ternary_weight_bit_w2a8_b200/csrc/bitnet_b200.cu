@@ -118,8 +118,8 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
-struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma"
-    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1;
+struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns"
+    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0;
 };
 
 const GemvTune &gemv_tune() {
@@ -127,7 +127,8 @@ const GemvTune &gemv_tune() {
     static std::once_flag once;
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
-        if (e != nullptr) sscanf(e, "%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma);
+        if (e != nullptr)
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma, &t.ns);
     });
     return t;
 }
@@ -203,37 +204,41 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 
-// TMA GEMV variants: (warps per CTA, boxes in flight per warp)
+// TMA GEMV variants: (warps per CTA, most boxes in flight per warp); the
+// ring depth of a launch is the smaller of the latter and what its items need
 constexpr int kTmaNumCfg = 5;
 constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
-// Kernel of (mode, variant, tokens per launch).  Several tokens (MT = 2, 4, 8)
-// are compiled for the 8 x 4 and 16 x 2 variants only; slot in the
-// shared-memory opt-in table: xmode * 11 + (MT == 1 ? cfg : 5 + 2 * log2(MT / 2) + (cfg == 2)).
+// Kernel of (mode, warps, tokens per launch).  int8 activations: one token on
+// 4, 8, 12 or 16 warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps.  bf16
+// activations quantised in the kernel: one token only (a batch is quantised
+// once beforehand and takes the int8 kernels).  Slot in the shared-memory
+// opt-in table: MT == 1 ? xmode * 10 + W / 4 - 1 : 4 + 2 * log2(MT / 2) + (W == 16); -1 if none.
 int tma_kernel_slot(int xmode, int cfg, int mt) {
-    const int base = mt == 1 ? cfg : 5 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (cfg == 2 ? 1 : 0);
-    return xmode * 11 + base;
+    const int W = kTmaCfg[cfg][0];
+    if (mt == 1) return xmode * 10 + W / 4 - 1;
+    if (xmode != 0 || (W != 8 && W != 16)) return -1;
+    return 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
 }
 
 TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
-    static const TmaKernel table[22] = {
-        gemv_tma_kernel<0, 8, 4, 1>, gemv_tma_kernel<0, 12, 3, 1>, gemv_tma_kernel<0, 16, 2, 1>,
-        gemv_tma_kernel<0, 8, 2, 1>, gemv_tma_kernel<0, 4, 4, 1>,
-        gemv_tma_kernel<0, 8, 4, 2>, gemv_tma_kernel<0, 16, 2, 2>, gemv_tma_kernel<0, 8, 4, 4>,
-        gemv_tma_kernel<0, 16, 2, 4>, gemv_tma_kernel<0, 8, 4, 8>, gemv_tma_kernel<0, 16, 2, 8>,
-        gemv_tma_kernel<1, 8, 4, 1>, gemv_tma_kernel<1, 12, 3, 1>, gemv_tma_kernel<1, 16, 2, 1>,
-        gemv_tma_kernel<1, 8, 2, 1>, gemv_tma_kernel<1, 4, 4, 1>,
-        gemv_tma_kernel<1, 8, 4, 2>, gemv_tma_kernel<1, 16, 2, 2>, gemv_tma_kernel<1, 8, 4, 4>,
-        gemv_tma_kernel<1, 16, 2, 4>, gemv_tma_kernel<1, 8, 4, 8>, gemv_tma_kernel<1, 16, 2, 8>};
-    return table[tma_kernel_slot(xmode, cfg, mt)];
+    static const TmaKernel table[14] = {
+        gemv_tma_kernel<0, 4, 1>, gemv_tma_kernel<0, 8, 1>, gemv_tma_kernel<0, 12, 1>, gemv_tma_kernel<0, 16, 1>,
+        gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 16, 4>,
+        gemv_tma_kernel<0, 8, 8>, gemv_tma_kernel<0, 16, 8>,
+        gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>};
+    const int slot = tma_kernel_slot(xmode, cfg, mt);
+    return slot < 0 ? nullptr : table[slot];
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
 size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    size_t &slot = dev->tma_max_dyn[tma_kernel_slot(xmode, cfg, mt)];
+    const int si = tma_kernel_slot(xmode, cfg, mt);
+    if (si < 0) return 0;
+    size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
         TmaKernel kern = tma_kernel_for(xmode, cfg, mt);
         cudaFuncAttributes fa;
@@ -245,21 +250,21 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
     return slot;
 }
 
-// Plan of the M = 1 TMA GEMV, from the shape and B200 reference figures only
-// (148 SMs, 228 KB of shared memory per SM), so that the workspace a shape
-// needs does not depend on the device that runs it.
+// Plan of the TMA GEMV, from the shape and B200 reference figures only (148
+// SMs, 227 KB of shared memory per CTA), so that what a shape needs does not
+// depend on the device that runs it.
 struct TmaPlan {
     bool use;
-    int cfg, slices, max_blocks, grid, max_parts;
+    int cfg, slices, max_blocks, grid;
+    int ns;            // ring depth per warp
     int mt;            // tokens per launch (1, 2, 4, 8)
-    int64_t ipc;       // > 0: split mode
     size_t smem;
-    int64_t ws_bytes;  // split mode: int32 parts and the BitLinear scale
+    int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
 };
 
 TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
-    constexpr size_t kRefSmemPerSM = 233472, kRefCtaReserve = 1024, kRefSmemOptin = 232448;
+    constexpr size_t kRefSmemOptin = 232448;
     TmaPlan p{};
     const int tune = gemv_tune().tma;
     if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
@@ -267,42 +272,30 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     const int64_t row_bytes = packed_row_bytes(K);
     const int64_t nblocks = ceil_div(N, kTmaRows);
     p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
-    // variant (measured on B200 over the sweep and large shapes): 16 warps x 2
-    // boxes in general, 12 x 3 for rows of K >= 16384, 8 x 4 below 3 MB
+    // variant (measured on B200 over sequences of different shapes, as in a
+    // decode step): 16 x 2, and 12 x 3 for rows of K >= 16384.  Variants that
+    // let two CTAs share an SM win on a shape repeated alone but lose in a
+    // mixed sequence, where the scheduler can then stack two CTAs of one
+    // launch on an SM.
     if (tune >= 1 && tune <= kTmaNumCfg)
         p.cfg = tune - 1;
     else
-        p.cfg = N * row_bytes < (3ll << 20) ? 0 : (p.slices >= 32 ? 1 : 2);
-    if (p.mt > 1 && p.cfg != 0) p.cfg = 2;  // several tokens: 8 x 4 or 16 x 2 only
+        p.cfg = p.slices >= 32 ? 1 : 2;
+    if (p.mt > 1 && kTmaCfg[p.cfg][0] != 8 && kTmaCfg[p.cfg][0] != 16) p.cfg = 2;  // several tokens: 8 or 16 warps
     const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
-    // resident CTAs per SM for the block-strided layout (accumulator slots are small)
-    const size_t base_smem = gemv_tma_smem_bytes(W, NS, p.slices, 1, p.mt);
-    int per_sm = (int)(kRefSmemPerSM / (base_smem + kRefCtaReserve));
-    if (per_sm > 2048 / (W * 32)) per_sm = 2048 / (W * 32);
-    if (per_sm < 1) return p;
+    // at most one CTA per SM per launch (BITNET_GEMV_TUNE's ctas field
+    // overrides): each SM keeps room for a CTA of the next launch, which then
+    // starts and requests its weights while this one finishes
+    const int per_sm = gemv_tune().ctas > 0 ? gemv_tune().ctas : 1;
     const int64_t gmax = (int64_t)kRefSMs * per_sm;
-    // split mode when whole row blocks per CTA would leave CTAs idle or uneven
-    // (more than 15 % above the mean), for problems large enough to pay the
-    // fixup launch (>= 4 MB of weights)
-    const int64_t g_strided = nblocks < gmax ? nblocks : gmax;
-    const double mean = (double)nblocks / (double)gmax, worst = (double)ceil_div(nblocks, g_strided);
-    // (measured on B200: the fixup launch costs more than the balance gains for
-    // every shape tried, so split mode is used only when asked for)
-    (void)mean;
-    (void)worst;
-    const bool want_split = gemv_tune().S == 1 && p.mt == 1;
-    if (want_split) {
-        const int64_t items = nblocks * p.slices;
-        p.ipc = ceil_div(items, gmax);
-        p.grid = (int)ceil_div(items, p.ipc);
-        p.max_blocks = (int)(ceil_div(p.ipc, p.slices) + 1);
-        p.max_parts = (int)(ceil_div(p.slices, p.ipc) + 1);
-        p.ws_bytes = round_up(nblocks * p.max_parts * kTmaRows * 4, 256) + 256;
-    } else {
-        p.grid = (int)g_strided;
-        p.max_blocks = (int)ceil_div(nblocks, g_strided);
-    }
-    p.smem = gemv_tma_smem_bytes(W, NS, p.slices, p.max_blocks, p.mt);
+    p.grid = (int)(nblocks < gmax ? nblocks : gmax);
+    p.max_blocks = (int)ceil_div(nblocks, p.grid);
+    // ring depth: no more boxes per warp than its items (a small launch then
+    // needs little shared memory and leaves room beside it)
+    const int64_t ipw = ceil_div((int64_t)p.max_blocks * p.slices, W);
+    p.ns = (int)(ipw < NS ? (ipw < 1 ? 1 : ipw) : NS);
+    if (gemv_tune().ns > 0) p.ns = gemv_tune().ns < NS ? gemv_tune().ns : NS;
+    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_blocks, p.mt);
     if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
     p.use = true;
     return p;
@@ -310,7 +303,9 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
 
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
-                    const TmaPlan &tp, void *ws, cudaStream_t st) {
+                    const TmaPlan &tp, cudaStream_t st) {
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
+    if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
     if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
@@ -323,7 +318,6 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
                              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return BITNET_ERR_CUDA;
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
     // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
     // makes one wait run out, exercising the device-timeout path
     static std::atomic<int> stall_once{-1};
@@ -344,20 +338,13 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.blk_begin = 0;
     a.nblocks = ceil_div(N, kTmaRows);
     a.max_blocks_cta = tp.max_blocks;
+    a.ns = tp.ns;
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
     a.s_act = s_act;
     a.test_stall = test_stall;
-    a.ipc = tp.ipc;
-    a.max_parts = tp.max_parts;
-    if (tp.ipc > 0) {
-        a.parts = static_cast<int32_t *>(ws);
-        a.s_out = reinterpret_cast<float *>(static_cast<char *>(ws) + tp.ws_bytes - 256);
-    }
-    int rc = launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
-    if (rc != BITNET_OK || tp.ipc == 0) return rc;
-    return launched(launch_pdl(gemv_tma_fixup_kernel, dim3(grid_for(N, 256, dev->sm_count)), dim3(256), (size_t)0, st, a));
+    return launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
 }
 
 // xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
@@ -368,7 +355,7 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     {
         const TmaPlan tp = tma_plan(M, N, K);
         if (tp.use && ldq == K)
-            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, ws, st);
+            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, st);
     }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();

@@ -26,7 +26,7 @@
 //     the block's item count writes the 32 results.
 //   - Every mbarrier wait is bounded in time.  A warp that gives up records
 //     BITNET_ERR_DEVICE_TIMEOUT, waits (bounded) for its own boxes in flight and
-//     returns; that row block's outputs are then left unwritten.
+//     stops; that row block's outputs are then left unwritten.
 //   - Programmatic dependent launch as in gemv.cuh: the first boxes of every
 //     warp are requested before griddepcontrol.wait.
 #pragma once
@@ -54,13 +54,7 @@ struct GemvTmaArgs {
     int64_t blk_begin;    // first row block of this launch
     int64_t nblocks;      // row blocks of this launch
     int max_blocks_cta;   // accumulator slots per CTA
-    // split mode (ipc > 0): CTA c takes items [c * ipc, (c + 1) * ipc) of the
-    // global (row block, slice) list and writes one int32 part per row block it
-    // touches to parts[block][c - first CTA of the block][32]
-    int64_t ipc;
-    int max_parts;        // parts per row block
-    int32_t *parts;
-    float *s_out;         // BitLinear split mode: the activation scale, for the fixup
+    int ns;               // ring depth per warp: boxes in flight
     int32_t *y_i32;       // [M, N] int32 result
     uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
     const float *gamma;   // weight scale (BitLinear)
@@ -69,7 +63,7 @@ struct GemvTmaArgs {
 };
 
 // Dynamic shared memory of a launch: ring of warps x stages boxes, linear
-// activations, per-row-block accumulators and counters, mbarriers.
+// activations, per-row-block accumulators and counters, slice sums, mbarriers.
 __host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta,
                                                       int tokens = 1) {
     return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes +
@@ -125,6 +119,8 @@ __device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *map, 
         : "memory");
 }
 
+// ------------------------------------------------------------------ staging
+
 // Adds up the 16-byte piece p of this lane into its K-slice's activation sum:
 // a warp stages 32 consecutive pieces (p = 32 w' + lane), exactly one slice of
 // 512 k, so one warp reduction gives the slice's sum.
@@ -157,37 +153,17 @@ __device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, int *qslice, const
 // arithmetic as quant_act_kernel), slice sums as above.  Returns the scale.
 __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, float *red, const uint16_t *xrow,
                                                  int64_t K, int64_t kq) {
-    constexpr int kHeld = 4;
     const bool vec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
-    const int64_t npieces = ceil_div(K, 16), qpieces = kq / 16;
-    uint4 held[kHeld][2];
+    const int64_t npieces = ceil_div(K, 16);
     float amax = 0.0f;
-#pragma unroll
-    for (int h = 0; h < kHeld; ++h) {
-        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
-        if (p < npieces) {
-            load_x16(xrow, K, p, vec, held[h][0], held[h][1]);
-            amax = amax16(held[h][0], held[h][1], amax);
-        }
-    }
-    for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < npieces; p += blockDim.x) {
+    for (int64_t p = threadIdx.x; p < npieces; p += blockDim.x) {
         uint4 lo, hi;
         load_x16(xrow, K, p, vec, lo, hi);
         amax = amax16(lo, hi, amax);
     }
     amax = block_reduce(amax, [](float u, float v) { return fmaxf(u, v); }, red);
     const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
-#pragma unroll
-    for (int h = 0; h < kHeld; ++h) {
-        const int64_t p = threadIdx.x + (int64_t)h * blockDim.x;
-        if (p < qpieces) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (p < npieces) quant16(held[h][0], held[h][1], sc, v);
-            *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
-            slice_sum(qslice, p, v);
-        }
-    }
-    for (int64_t p = threadIdx.x + (int64_t)kHeld * blockDim.x; p < qpieces; p += blockDim.x) {
+    for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (p < npieces) {
             uint4 lo, hi;
@@ -200,62 +176,54 @@ __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, floa
     return sc;
 }
 
-template <int XMODE, int W, int NS, int MT>
-__global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
+// ------------------------------------------------------------------ kernel
+
+// Resident CTAs the register budget leaves room for: two for the 8-warp and
+// smaller variants (up to 4 tokens), so that the next launch's CTAs can start
+// (and request their weights) on an SM while this launch is finishing there.
+template <int W, int MT>
+constexpr int gemv_tma_min_blocks() { return (W <= 8 && MT <= 4) ? 2 : 1; }
+
+template <int XMODE, int W, int MT>
+__global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
+    gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
     static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8, "tokens per launch");
+    static_assert(XMODE == 0 || MT == 1, "bf16 activations: one token per launch");
     extern __shared__ uint8_t smem_raw[];
     __shared__ float red[32];
-    // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8 rows
-    // of 128 bytes); computed on the shared-window address so that every
+    // the descriptor fetch is the first long latency of the launch: start it now
+    if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+    const int ns = a.ns, slices = a.slices;
+    const int64_t cid = blockIdx.x, ncl = gridDim.x;  // row blocks cid, cid + ncl, ...
+    const int64_t kq = (int64_t)slices * kTmaSliceK;
+
+    // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8
+    // rows of 128 bytes), computed on the shared-window address so that every
     // pointer below stays a shared-memory pointer
     uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * NS * kTmaBoxBytes);   // [MT][kq]
-    const int64_t kq = (int64_t)a.slices * kTmaSliceK;
+    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kTmaBoxBytes);   // [MT][kq]
     int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][32]
-    int *done = accs + a.max_blocks_cta * MT * kTmaRows;
+    int *done = accs + a.max_blocks_cta * MT * kTmaRows;                       // [slot] items done
     int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
     uint64_t *bars =
-        reinterpret_cast<uint64_t *>(qslice + MT * a.slices + ((a.max_blocks_cta + MT * a.slices) & 1));
+        reinterpret_cast<uint64_t *>(qslice + MT * slices + ((a.max_blocks_cta + MT * slices) & 1));
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int slices = a.slices;
-    const bool split = a.ipc > 0;  // (single-token launches only)
-    // this CTA's items, in (row block, slice) order; `bstep` is the distance
-    // between consecutive row blocks of the CTA
-    int64_t cta_begin, items, first_block, bstep;
-    if (split) {
-        const int64_t total = a.nblocks * slices;
-        cta_begin = min(total, (int64_t)blockIdx.x * a.ipc);
-        items = min(total, cta_begin + a.ipc) - cta_begin;
-        first_block = cta_begin / slices;
-        bstep = 1;
-    } else {
-        const int64_t nb_cta = a.nblocks > blockIdx.x ? ceil_div(a.nblocks - blockIdx.x, gridDim.x) : 0;
-        cta_begin = 0;
-        items = nb_cta * slices;
-        first_block = blockIdx.x;
-        bstep = gridDim.x;
-    }
-    const int j0 = (int)(split ? cta_begin - first_block * slices : 0);  // slice of the CTA's first item
-    const int nslots = (int)((j0 + items + slices - 1) / slices);        // row blocks touched
+    // this CTA's items, in (row block, slice) order
+    const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
+    const int64_t items = nb_cta * slices;
+    const int nslots = (int)nb_cta;
     // this warp's items: a contiguous range of the CTA's items
     const int64_t ipw = ceil_div(items, W);
     const int64_t it_begin = min(items, warp * ipw);
     const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
-    uint64_t *mybar = bars + warp * NS;
-    uint8_t *myring = ring + warp * NS * kTmaBoxBytes;
+    uint64_t *mybar = bars + warp * ns;
+    uint8_t *myring = ring + warp * ns * kTmaBoxBytes;
 
-    if (threadIdx.x < W * NS) mbar_init(&bars[threadIdx.x], 1);
-    for (int i = threadIdx.x; i < nslots * MT * kTmaRows; i += blockDim.x) accs[i] = 0;
-    for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    __syncthreads();
-
-    // cursor over the warp's items: (slot, slice); row block = first_block + slot * bstep
-    const int64_t p0 = j0 + it_begin;
-    int islot = (int)(p0 / slices), ij = (int)(p0 - (int64_t)(p0 / slices) * slices);
+    // cursor over the warp's items: (slot, slice); row block = cid + slot * ncl
+    int islot = (int)(it_begin / slices), ij = (int)(it_begin - (int64_t)islot * slices);
     auto issue_next = [&](int s) {
-        const int64_t row0 = (a.blk_begin + first_block + (int64_t)islot * bstep) * kTmaRows;
+        const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * kTmaRows;
         mbar_arrive_expect_tx(&mybar[s], kTmaBoxBytes);
         tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
         if (++ij == slices) {
@@ -263,9 +231,13 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
             ++islot;
         }
     };
-    // weights do not depend on the previous kernel: request them before waiting for it
+    // weights do not depend on the previous kernel: request them before waiting
+    // for it.  A warp's ring and barriers are its own, so lane 0 sets them up
+    // and issues without waiting for the rest of the CTA.
     if (lane == 0) {
-        for (int s = 0; s < NS && s < n_items; ++s) {
+        for (int s = 0; s < ns; ++s) mbar_init(&mybar[s], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < ns && s < n_items; ++s) {
             if (s == 0 && warp == 0 && a.test_stall) {  // skip the request: nothing completes this stage
                 if (++ij == slices) {
                     ij = 0;
@@ -276,6 +248,8 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
             issue_next(s);
         }
     }
+    for (int i = threadIdx.x; i < nslots * MT * kTmaRows; i += blockDim.x) accs[i] = 0;
+    for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
     pdl_launch_dependents();
     pdl_wait();
 
@@ -296,14 +270,12 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
             for (int j = threadIdx.x; j < slices; j += blockDim.x) qst[j] = 0;
         }
     }
-    if (split && XMODE == 1 && a.s_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.s_out = sc[0];
     __syncthreads();
     float f[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         f[t] = 0.0f;
-        if (!split && t < a.M && a.y_bf16 != nullptr)
-            f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
+        if (t < a.M && a.y_bf16 != nullptr) f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
     }
 
     int acc[MT][4], corr[MT];
@@ -311,7 +283,7 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
     int ncontrib = 0;
     // folds this warp's partial sums of slot `sl` into shared memory; the warp
-    // completing the slot's items writes its results (split mode: its part)
+    // completing the slot's items writes its results
     auto flush = [&](int sl) {
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
@@ -320,26 +292,16 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
         }
         __threadfence_block();
         __syncwarp();
-        const int64_t blk = first_block + (int64_t)sl * bstep;
-        int expected = slices;
-        if (split) {
-            const int64_t lo = max(cta_begin, blk * slices), hi = min(cta_begin + items, (blk + 1) * slices);
-            expected = (int)(hi - lo);
-        }
         int fin = 0;
-        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == expected);
+        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == slices);
         fin = __shfl_sync(0xffffffffu, fin, 0);
         if (fin) {
             __threadfence_block();
-            const int64_t gb = a.blk_begin + blk;
-            const int64_t n = gb * kTmaRows + lane;
+            const int64_t n = (a.blk_begin + cid + (int64_t)sl * ncl) * kTmaRows + lane;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
                 const int tot = atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], 0);
-                if (split) {
-                    const int64_t first_cta = (gb * slices) / a.ipc;
-                    a.parts[(gb * a.max_parts + (blockIdx.x - first_cta)) * kTmaRows + lane] = tot;
-                } else if (t < a.M && n < a.N) {
+                if (t < a.M && n < a.N) {
                     if (a.y_bf16 != nullptr)
                         a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
                     else
@@ -353,15 +315,16 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
     };
 
     // consume cursor
-    int cslot = (int)(p0 / slices), cj = (int)(p0 - (int64_t)(p0 / slices) * slices);
+    int cslot = (int)(it_begin / slices), cj = (int)(it_begin - (int64_t)cslot * slices);
+    int s = 0;
+    uint32_t phase = 0;
     for (int n = 0; n < n_items; ++n) {
-        const int s = n % NS;
-        if (!mbar_wait_bounded(&mybar[s], (uint32_t)(n / NS) & 1u)) {
+        if (!mbar_wait_bounded(&mybar[s], phase)) {
             if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
-            // wait (bounded) for this warp's other boxes still in flight, then leave
-            for (int d = 1; d < NS && n + d < n_items; ++d)
-                mbar_wait_bounded(&mybar[(n + d) % NS], (uint32_t)((n + d) / NS) & 1u);
-            return;
+            // wait (bounded) for this warp's other boxes still in flight, then stop
+            for (int d = 1; d < ns && n + d < n_items; ++d)
+                mbar_wait_bounded(&mybar[(n + d) % ns], (uint32_t)((n + d) / ns) & 1u);
+            break;
         }
         const uint8_t *row = myring + s * kTmaBoxBytes + lane * kTmaSliceBytes;
         const int8_t *qk = qlin + cj * kTmaSliceK;
@@ -404,31 +367,16 @@ __global__ void __launch_bounds__(W * 32, 1) gemv_tma_kernel(const __grid_consta
 #pragma unroll
         for (int t = 0; t < MT; ++t) corr[t] += qslice[t * slices + cj];
         __syncwarp();
-        if (lane == 0 && n + NS < n_items) issue_next(s);
+        if (lane == 0 && n + ns < n_items) issue_next(s);
+        if (++s == ns) {
+            s = 0;
+            phase ^= 1u;
+        }
         if (++cj == slices || n + 1 == n_items) {
             flush(cslot);
             cj = 0;
             ++cslot;
         }
-    }
-}
-
-// Split-mode fixup: y[n] = sum of the int32 parts of n's row block, in CTA
-// order, then the int32 or BitLinear epilogue.
-__global__ void __launch_bounds__(256) gemv_tma_fixup_kernel(const GemvTmaArgs a) {
-    pdl_wait();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    float f = 0.0f;
-    if (a.y_bf16 != nullptr) f = __fdiv_rn(*a.gamma, *a.s_out);
-    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < a.N; n += stride) {
-        const int64_t b = n / kTmaRows;
-        const int64_t c0 = (b * a.slices) / a.ipc, c1 = ((b + 1) * a.slices - 1) / a.ipc;
-        int t = 0;
-        for (int64_t c = c0; c <= c1; ++c) t += a.parts[(b * a.max_parts + (c - c0)) * kTmaRows + (n % kTmaRows)];
-        if (a.y_bf16 != nullptr)
-            a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)t, f));
-        else
-            a.y_i32[n] = t;
     }
 }
 

@@ -41,7 +41,8 @@ print(json.dumps({"status": status, "again": again, "exact_after": exact, "secon
 """
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("tune", [None, "0,0,0,0,-1,0,3"])  # the planner's variant; 16 warps
+def test_bounded_wait_reports_timeout_and_context_survives(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -49,6 +50,8 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     env = dict(os.environ)
     env["BITNET_TEST_STALL"] = "1"
     env.pop("BITNET_GEMV_TUNE", None)
+    if tune is not None:
+        env["BITNET_GEMV_TUNE"] = tune
     r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + CHILD], env=env,
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
