@@ -2,6 +2,7 @@
 // include/bitnet_b200.h): argument checks, plan selection and launches.
 // All kernels are in the headers included below; this is the library's single
 // translation unit, so file-scope device state (the error word) is shared.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
@@ -37,7 +38,7 @@ struct DeviceInfo {
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
     size_t tma_max_dyn[22] = {};  // dynamic shared memory opted into by each TMA GEMV variant
-    bool tc_attr_set[8] = {false, false, false, false, false, false, false, false};
+    bool tc_attr_set[10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
     OccEntry occ[kOccCache];     // resident CTAs per SM by (instantiation, shared memory)
@@ -449,56 +450,79 @@ int noalloc_scratch(void **out) {
 }
 
 // ------------------------------------------------------------------ tcgen05 GEMM (M > 1)
-constexpr int kTcBNs[4] = {256, 128, 96, 64};
+// Token-tile widths (UMMA N) of the tensor-core GEMM.
+constexpr int kTcNumBT = 5;
+constexpr int kTcBTs[kTcNumBT] = {256, 128, 64, 32, 16};
 using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
-// Operand rings per tile width: (activation/code stages, packed stages).  The
-// widest tile runs one CTA per SM; the narrower ones keep two CTAs per SM
-// (shared memory <= 113 KB, tensor memory <= 256 columns each).  A 4 + 2 ring
-// for the widest tile measured slower on B200 than 3 + 3 (91.5 vs 87.0 us at
-// M = 2048, N = 13824, K = 2560).
-TcKernel tc_kernel_for(int bn_idx, bool bf16, size_t *smem) {
-    static const TcKernel k[8] = {gemm_w2a8_tc_kernel<256, false, 3, 3>, gemm_w2a8_tc_kernel<128, false, 3, 3>,
-                                  gemm_w2a8_tc_kernel<96, false, 3, 3>,  gemm_w2a8_tc_kernel<64, false, 3, 3>,
-                                  gemm_w2a8_tc_kernel<256, true, 3, 3>,  gemm_w2a8_tc_kernel<128, true, 3, 3>,
-                                  gemm_w2a8_tc_kernel<96, true, 3, 3>,   gemm_w2a8_tc_kernel<64, true, 3, 3>};
-    static const size_t sz[4] = {TcSmem<256, 3, 3>::kBytes + 1024, TcSmem<128, 3, 3>::kBytes + 1024,
-                                 TcSmem<96, 3, 3>::kBytes + 1024, TcSmem<64, 3, 3>::kBytes + 1024};
-    *smem = sz[bn_idx];
-    return k[(bf16 ? 4 : 0) + bn_idx];
+// Rings (activation, code, packed stages) per token-tile width.  The widest
+// tile runs one CTA per SM (tensor memory 256 + 4 x 32 columns -> 512); the
+// others request at least 80 KB of shared memory so that at most two CTAs
+// share an SM and their tensor-memory allocations (256 columns) always fit.
+TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
+    static const TcKernel k[2 * kTcNumBT] = {
+        gemm_w2a8_tc_kernel<256, false, 4, 4, 6>, gemm_w2a8_tc_kernel<128, false, 4, 4, 6>,
+        gemm_w2a8_tc_kernel<64, false, 6, 4, 6>,  gemm_w2a8_tc_kernel<32, false, 8, 4, 8>,
+        gemm_w2a8_tc_kernel<16, false, 8, 4, 8>,  gemm_w2a8_tc_kernel<256, true, 4, 4, 6>,
+        gemm_w2a8_tc_kernel<128, true, 4, 4, 6>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
+        gemm_w2a8_tc_kernel<32, true, 8, 4, 8>,   gemm_w2a8_tc_kernel<16, true, 8, 4, 8>};
+    static const size_t raw[kTcNumBT] = {TcSmem<256, 4, 4, 6>::kBytes, TcSmem<128, 4, 4, 6>::kBytes,
+                                         TcSmem<64, 6, 4, 6>::kBytes, TcSmem<32, 8, 4, 8>::kBytes,
+                                         TcSmem<16, 8, 4, 8>::kBytes};
+    const size_t need = raw[bt_idx] + 1024;  // + alignment slack
+    *smem = (bt_idx == 0 || need >= 80 * 1024) ? need : 80 * 1024;
+    return k[(bf16 ? kTcNumBT : 0) + bt_idx];
 }
 
-// Weight rows per tile: the largest tile that still gives every SM a tile.
-int tc_bn_index(int64_t M, int64_t N, int sm_count) {
-    const int64_t mt = ceil_div(M, kTcBM);
-    for (int i = 0; i < 4; ++i)
-        if (mt * ceil_div(N, kTcBNs[i]) >= sm_count) return i;
-    return 3;
-}
-
-// Tile width and K-split of the tensor-core GEMM.  Computed for the B200's
-// 148 SMs whatever the device, so the workspace a shape needs is fixed.
+// Token-tile width and K-split of the tensor-core GEMM, from a small cost
+// model of the kernel on the B200's 148 SMs (so the workspace a shape needs
+// is fixed whatever the device): a stage of 128 k takes
+// max(MMA time ~0.37 us x BT / 256, decode ~0.15 us); a CTA adds ~1.5 us of
+// set-up and epilogue; a K-split adds the zeroing launch and the reduce-add
+// stores (~2.5 us).  Candidates: token tiles from the smallest that holds M
+// (at most 256) down to 16, splits 1..16.
 struct TcPlan {
-    int bn_idx, S, sps;
+    int bt_idx, S, sps;
 };
 
 TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
     TcPlan p{};
     const GemvTune &tn = gemv_tune();
-    p.bn_idx = tc_bn_index(M, N, kRefSMs);
-    if (tn.R < 0 && -tn.R <= 4) p.bn_idx = -tn.R - 1;  // tuning override: R = -1..-4 picks the tile width
     const int nk = (int)(k_pad(K) / kTcBK);
-    const int64_t tiles = ceil_div(M, kTcBM) * ceil_div(N, kTcBNs[p.bn_idx]);
-    int S = 1;
-    if (tiles * 2 <= kRefSMs && nk >= 8) {
-        S = (int)(kRefSMs / tiles);
-        if (S > nk / 4) S = nk / 4;
-        if (S < 1) S = 1;
+    const int64_t nt = ceil_div(N, kTcRows);
+    int first = kTcNumBT - 1;
+    while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else 256
+    double best = 1e30;
+    for (int i = first; i < kTcNumBT; ++i) {
+        const int BT = kTcBTs[i];
+        const int64_t tiles = nt * ceil_div(M, BT);
+        const int64_t slots = (int64_t)kRefSMs * (BT == 256 ? 1 : 2);
+        const double stage_us = std::max(0.37 * BT / 256.0, 0.15);
+        for (int S = 1; S <= 16 && S <= nk; ++S) {
+            const int sps = (int)ceil_div(nk, S);
+            const int Se = (int)ceil_div(nk, sps);
+            if (Se != S) continue;
+            const int64_t waves = ceil_div(tiles * S, slots);
+            const double t = (double)waves * (sps * stage_us + 1.5) + (S > 1 ? 2.5 : 0.0);
+            if (t < best * 0.999) {
+                best = t;
+                p.bt_idx = i;
+                p.S = S;
+                p.sps = sps;
+            }
+        }
     }
-    if (tn.S > 0) S = tn.S < nk ? tn.S : nk;  // tuning override
-    p.sps = (int)ceil_div(nk, S);
-    p.S = (int)ceil_div(nk, p.sps);
+    // tuning overrides: R = -1..-5 picks the token tile, S the split count
+    if (tn.R < 0 && -tn.R <= kTcNumBT) p.bt_idx = -tn.R - 1;
+    if (tn.S > 0) {
+        const int S = tn.S < nk ? tn.S : nk;
+        p.sps = (int)ceil_div(nk, S);
+        p.S = (int)ceil_div(nk, p.sps);
+    } else if (tn.R < 0) {
+        p.S = 1;
+        p.sps = nk;
+    }
     return p;
 }
 
@@ -507,14 +531,14 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
                    const TcPlan &tp, int reduce, cudaStream_t st) {
     if (tensor_map_encoder() == nullptr) return BITNET_ERR_CUDA;
-    const int bi = tp.bn_idx;
-    const int BN = kTcBNs[bi];
+    const int bi = tp.bt_idx;
+    const int BT = kTcBTs[bi];
     const bool bf16 = y_bf16 != nullptr;
     size_t smem = 0;
     TcKernel kern = tc_kernel_for(bi, bf16, &smem);
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
-        bool &set = dev->tc_attr_set[(bf16 ? 4 : 0) + bi];
+        bool &set = dev->tc_attr_set[(bf16 ? kTcNumBT : 0) + bi];
         if (!set) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return BITNET_ERR_CUDA;
@@ -525,7 +549,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t gstride[1] = {(cuuint64_t)lda};
-        const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBM};
+        const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)BT};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(q), gdim, gstride, box,
                                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -536,7 +560,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         const int64_t row_bytes = packed_row_bytes(K);
         const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
         const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-        const cuuint32_t box[2] = {32u, (cuuint32_t)BN};
+        const cuuint32_t box[2] = {32u, (cuuint32_t)kTcRows};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
                                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
@@ -553,11 +577,12 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     if (tma_store) {
         const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
         const cuuint64_t gstride[1] = {(cuuint64_t)(N * esize)};
-        const cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 32u};
+        // boxes of 32 weight rows (inner) x up to 32 tokens, unswizzled
+        const cuuint32_t box[2] = {(cuuint32_t)kTcBox, (cuuint32_t)(BT < kTcBox ? BT : kTcBox)};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&ymap, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_INT32, 2,
                                  ybase, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             tma_store = 0;
     }
@@ -573,7 +598,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.tma_store = tma_store;
     a.sps = tp.sps;
     a.reduce = reduce;
-    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)ceil_div(M, kTcBM), (unsigned)tp.S);
+    const dim3 grid((unsigned)ceil_div(N, kTcRows), (unsigned)ceil_div(M, BT), (unsigned)tp.S);
     return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, ymap, a));
 }
 

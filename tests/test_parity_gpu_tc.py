@@ -2,8 +2,8 @@
 
 Ragged shapes (M, N not multiples of the tile, K not a multiple of the
 128-byte stage or of 16, which makes the library repack the activations), every
-tile width (forced in child processes through BITNET_GEMV_TUNE, read once per
-process), int32 and BitLinear bf16 outputs.
+token-tile width with and without a K-split (forced in child processes through
+BITNET_GEMV_TUNE, read once per process), int32 and BitLinear bf16 outputs.
 """
 import json
 import os
@@ -75,20 +75,32 @@ import oracle
 import ternary_weight_bit_w2a8_b200 as bn
 from ternary_weight_bit_w2a8_b200 import synth
 out = {}
-for (M, N, K) in [(130, 300, 1000), (256, 520, 2560), (3, 1000, 384)]:
+for (M, N, K) in [(130, 300, 1000), (256, 520, 2560), (9, 1000, 384), (40, 129, 640), (300, 64, 4096)]:
     q, w = synth.uniform_int8_ternary(N, K, seed=M * N + K, M=M)
+    q[-1, :] = -128
     y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
     out[f"{M}x{N}x{K}"] = bool(np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w)))
+for (M, N, K) in [(33, 200, 1000), (260, 96, 512)]:
+    x, W = synth.bitlinear_inputs(M, N, K, seed=M)
+    g = oracle.absmean(W)
+    wt = oracle.ternarize(W, g)
+    yb = bn.bitnet_bitlinear(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16),
+                             bn.bitnet_pack_weights(torch.from_numpy(wt).cuda()),
+                             torch.tensor([float(g)], dtype=torch.float32, device="cuda"), N)
+    yr = oracle.bitlinear(x, wt, g)[0]
+    err = np.abs(yb.float().cpu().numpy().astype(np.float64) - yr)
+    out[f"bitlinear {M}x{N}x{K}"] = bool(np.where(np.abs(yr) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(yr)).all())
 torch.cuda.synchronize()
 out["device_error"] = bn.bitnet_get_device_error()
 print(json.dumps(out))
 """
 
 
-@pytest.mark.parametrize("tile", [1, 2, 3, 4])  # BN = 256, 128, 96, 64
-def test_tc_every_tile_width(tile):
+# token tile 1..5 = 256, 128, 64, 32, 16 tokens; S = K-splits (0: none when a tile is forced)
+@pytest.mark.parametrize("tile,S", [(1, 0), (2, 0), (3, 0), (4, 0), (5, 0), (1, 3), (3, 5), (5, 2)])
+def test_tc_every_tile_width(tile, S):
     env = dict(os.environ)
-    env["BITNET_GEMV_TUNE"] = f"0,-{tile},0,0,-1,0,-1"
+    env["BITNET_GEMV_TUNE"] = f"0,-{tile},0,0,-1,{S},-1"
     r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + CHILD], env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
