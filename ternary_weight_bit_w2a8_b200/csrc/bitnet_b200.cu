@@ -450,37 +450,41 @@ int noalloc_scratch(void **out) {
 }
 
 // ------------------------------------------------------------------ tcgen05 GEMM (M > 1)
-// Token-tile widths (UMMA N) of the tensor-core GEMM.
+// Token-tile widths (UMMA N) of the persistent tensor-core GEMM.
 constexpr int kTcNumBT = 5;
-constexpr int kTcBTs[kTcNumBT] = {256, 128, 64, 32, 16};
+constexpr int kTcBTs[kTcNumBT] = {192, 128, 64, 32, 16};
 using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
-// Rings (activation, code, packed stages) per token-tile width.  The widest
-// tile runs one CTA per SM (tensor memory 256 + 4 x 32 columns -> 512); the
-// others request at least 80 KB of shared memory so that at most two CTAs
-// share an SM and their tensor-memory allocations (256 columns) always fit.
+// Rings (activation, code, packed stages) per token-tile width.  The 192- and
+// 128-token variants take all 512 tensor-memory columns (2 accumulators + 4
+// code stages) and more than half an SM's shared memory, so one CTA per SM;
+// the narrower ones take 256 columns and at most two CTAs share an SM.
 TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
     static const TcKernel k[2 * kTcNumBT] = {
-        gemm_w2a8_tc_kernel<256, false, 4, 4, 6>, gemm_w2a8_tc_kernel<128, false, 4, 4, 6>,
+        gemm_w2a8_tc_kernel<192, false, 4, 4, 6>, gemm_w2a8_tc_kernel<128, false, 5, 4, 6>,
         gemm_w2a8_tc_kernel<64, false, 6, 4, 6>,  gemm_w2a8_tc_kernel<32, false, 8, 4, 8>,
-        gemm_w2a8_tc_kernel<16, false, 8, 4, 8>,  gemm_w2a8_tc_kernel<256, true, 4, 4, 6>,
-        gemm_w2a8_tc_kernel<128, true, 4, 4, 6>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
+        gemm_w2a8_tc_kernel<16, false, 8, 4, 8>,  gemm_w2a8_tc_kernel<192, true, 4, 4, 6>,
+        gemm_w2a8_tc_kernel<128, true, 5, 4, 6>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
         gemm_w2a8_tc_kernel<32, true, 8, 4, 8>,   gemm_w2a8_tc_kernel<16, true, 8, 4, 8>};
-    static const size_t raw[kTcNumBT] = {TcSmem<256, 4, 4, 6>::kBytes, TcSmem<128, 4, 4, 6>::kBytes,
+    static const size_t raw[kTcNumBT] = {TcSmem<192, 4, 4, 6>::kBytes, TcSmem<128, 5, 4, 6>::kBytes,
                                          TcSmem<64, 6, 4, 6>::kBytes, TcSmem<32, 8, 4, 8>::kBytes,
                                          TcSmem<16, 8, 4, 8>::kBytes};
-    const size_t need = raw[bt_idx] + 1024;  // + alignment slack
-    *smem = (bt_idx == 0 || need >= 80 * 1024) ? need : 80 * 1024;
+    *smem = raw[bt_idx] + 1024;  // + alignment slack
     return k[(bf16 ? kTcNumBT : 0) + bt_idx];
 }
 
 // Token-tile width and K-split of the tensor-core GEMM, from a small cost
-// model of the kernel on the B200's 148 SMs (so the workspace a shape needs
-// is fixed whatever the device): a stage of 128 k takes
-// max(MMA time ~0.37 us x BT / 256, decode ~0.15 us); a CTA adds ~1.5 us of
-// set-up and epilogue; a K-split adds the zeroing launch and the reduce-add
-// stores (~2.5 us).  Candidates: token tiles from the smallest that holds M
-// (at most 256) down to 16, splits 1..16.
+// model of the persistent kernel on the B200's 148 SMs (so the workspace a
+// shape needs is fixed whatever the device): an SM runs its work units one
+// after another; a stage of 128 k took about 0.4 us for every token-tile
+// width measured on B200 (the hand-over between decoders and tensor core
+// bounds it, not the MMA), so the model charges max(0.4 us, the MMA time);
+// the pipeline fill and the last epilogue add ~2 us.  A K-split is considered
+// only when the tiles do not fill the SMs; it adds a launch (~2.5 us) plus
+// the zeroing of the int32 output and one reduce-add pass over it per split,
+// each at ~1.4 TB/s (measured: a 2-way split of M = 2048, N = 13824 cost more
+// than the whole unsplit GEMM).  Candidates: token tiles from the smallest
+// that holds M (at most 192) down to 16, splits 1..16.
 struct TcPlan {
     int bt_idx, S, sps;
 };
@@ -492,19 +496,19 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     const int nk = (int)(k_pad(K) / kTcBK);
     const int64_t nt = ceil_div(N, kTcRows);
     int first = kTcNumBT - 1;
-    while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else 256
+    while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else the widest
     double best = 1e30;
     for (int i = first; i < kTcNumBT; ++i) {
         const int BT = kTcBTs[i];
         const int64_t tiles = nt * ceil_div(M, BT);
-        const int64_t slots = (int64_t)kRefSMs * (BT == 256 ? 1 : 2);
-        const double stage_us = std::max(0.37 * BT / 256.0, 0.15);
+        const double stage_us = std::max(0.41 * BT / 256.0, 0.40);
+        const double out_us = (double)M * (double)N * 4.0 / 1.4e6;  // one pass over the int32 output
         for (int S = 1; S <= 16 && S <= nk; ++S) {
+            if (S > 1 && tiles >= kRefSMs) break;
             const int sps = (int)ceil_div(nk, S);
-            const int Se = (int)ceil_div(nk, sps);
-            if (Se != S) continue;
-            const int64_t waves = ceil_div(tiles * S, slots);
-            const double t = (double)waves * (sps * stage_us + 1.5) + (S > 1 ? 2.5 : 0.0);
+            if (ceil_div(nk, sps) != S) continue;
+            const int64_t rounds = ceil_div(tiles * S, kRefSMs);
+            const double t = (double)rounds * sps * stage_us + 2.0 + (S > 1 ? 2.5 + (S + 1) * out_us : 0.0);
             if (t < best * 0.999) {
                 best = t;
                 p.bt_idx = i;
@@ -598,8 +602,14 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.tma_store = tma_store;
     a.sps = tp.sps;
     a.reduce = reduce;
-    const dim3 grid((unsigned)ceil_div(N, kTcRows), (unsigned)ceil_div(M, BT), (unsigned)tp.S);
-    return launched(launch_pdl(kern, grid, dim3(kTcThreads), smem, st, amap, pmap, ymap, a));
+    a.tiles_n = (int)ceil_div(N, kTcRows);
+    a.tiles_m = (int)ceil_div(M, BT);
+    a.splits = tp.S;
+    // persistent: one CTA per SM (or fewer, when there are fewer work units)
+    const int64_t units = (int64_t)a.tiles_n * a.tiles_m * a.splits;
+    if (units > (int64_t)1 << 30) return BITNET_ERR_UNSUPPORTED;  // work units are counted in int
+    const int grid = (int)(units < dev->sm_count ? units : dev->sm_count);
+    return launched(launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, amap, pmap, ymap, a));
 }
 
 // Copies int8 activations [M, K] into rows of K_pad bytes, zero-padded, so the

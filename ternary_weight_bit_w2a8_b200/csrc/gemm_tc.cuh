@@ -6,34 +6,40 @@
 // The pages have no M > 1 kernel: their GEMV handles M == 1 only (page "如何编
 // 译 BitNet W2A8 CUDA 内核并用 test.py 运行 GEMV 加速测试？", section 限制与注意
 // 事项).  Design: the ternary weights are the MMA's A operand and live in
-// tensor memory, so decoded weights never pass through shared memory.
-//   - CTA tile: 128 weight rows (UMMA M) x BT tokens (UMMA N) x 128 k per
-//     stage; the accumulator D[n, m] takes 128 TMEM lanes x BT columns.
-//   - Warp 0, one lane: TMA producer of two rings, each with full / empty
-//     mbarriers: activation tiles (int8 [BT tokens x 128 bytes], 128-byte
-//     swizzle: the canonical K-major B operand; SA stages) and packed weight
-//     tiles (layout v1, [128 rows x 32 bytes], 32-byte swizzle; SP stages).
-//     The first packed tiles are requested before griddepcontrol.wait (weights
-//     never depend on an earlier kernel).
-//   - Warps 2..5: decoders.  A thread owns one weight row (its warp's TMEM lane
-//     quarter).  Per stage the row's 8 packed words (128 k) become 32 words of
+// tensor memory, so decoded weights never pass through shared memory; the
+// kernel is persistent, one CTA per SM looping over work units.
+//   - Work unit: 128 weight rows (UMMA M) x BT tokens (UMMA N) x one K-split;
+//     units are dealt round-robin to the CTAs, weight-row tiles fastest.  A
+//     unit is done in stages of 128 k; its accumulator D[n, m] takes 128 TMEM
+//     lanes x BT columns, and two accumulators alternate so that one unit's
+//     epilogue overlaps the next unit's main loop.
+//   - Warp 0, one lane: TMA producer of two rings that run on across units,
+//     each with full / empty mbarriers: activation tiles (int8 [BT tokens x
+//     128 bytes], 128-byte swizzle: the canonical K-major B operand; SA stages)
+//     and packed weight tiles (layout v1, [128 rows x 32 bytes], 32-byte
+//     swizzle; SP stages).  The first packed tiles are requested before
+//     griddepcontrol.wait (weights never depend on an earlier kernel).
+//   - Warps 2..9: decoders, two groups of four that take alternate stages (a
+//     group's tensor-memory store latency hides behind the other group's
+//     work).  A thread owns one weight row (its warp's TMEM lane quarter).
+//     Per stage the row's 8 packed words (128 k) become 32 words of
 //     signed codes: (word >> 2j) & 0x03030303 gives the codes c of 4
 //     consecutive k, and ((c + 0x7F7F7F7F) ^ 0x80808080) is c - 1 in every
 //     byte with no carry between bytes.  One tcgen05.st writes the 32 words
 //     into a code stage of tensor memory (SC stages of 32 columns).
 //   - Warp 1: allocates tensor memory and, from one lane, issues per stage four
 //     K = 32 MMAs (A = codes in tensor memory, B = activations in shared
-//     memory, s8 x s8 -> s32); tcgen05.commit on per-stage mbarriers releases
-//     the activation and code stages.
-//   - After the last stage, warps 2..5 read the accumulators (tcgen05.ld: one
-//     weight row per thread, 16 tokens per load), keep int32 or scale by
-//     gamma / s_m to bf16, and stage 32-token x 32-row boxes in the freed
-//     activation ring for TMA stores; direct stores are the fallback when the
-//     output rows are not 16-byte strided.
-//   - Split-K (gridDim.z > 1, for problems with fewer tiles than SMs): each
-//     split covers a range of k stages and adds its int32 partial sums into a
-//     zeroed output with TMA reduce-add stores (integer adds: exact and
-//     order-free).
+//     memory, s8 x s8 -> s32) into the unit's accumulator; tcgen05.commit on
+//     per-stage mbarriers releases the activation and code stages, and on a
+//     per-accumulator mbarrier hands a finished unit to the epilogue.
+//   - Warps 10..13: epilogue.  They read an accumulator (tcgen05.ld: one weight
+//     row per thread, 16 tokens per load), keep int32 or scale by gamma / s_m
+//     to bf16, stage 32-token x 32-row boxes in shared memory for TMA stores
+//     (direct stores when the output rows are not 16-byte strided) and release
+//     the accumulator.
+//   - Split-K (for problems with fewer tiles than SMs): each split covers a
+//     range of k stages and adds its int32 partial sums into a zeroed output
+//     with TMA reduce-add stores (integer adds: exact and order-free).
 //   - Every mbarrier wait is bounded in time; a role that gives up records
 //     BITNET_ERR_DEVICE_TIMEOUT and raises a shared abort flag that stops the
 //     others; all roles then drain what they issued (bounded) and tensor
@@ -50,13 +56,18 @@ namespace bitnet {
 
 constexpr int kTcRows = 128;            // weight rows per tile (UMMA M)
 constexpr int kTcBK = 128;              // k per stage (bytes of an activation row)
-constexpr int kTcThreads = 192;         // 6 warps
+constexpr int kTcDecGroups = 2;        // decoder groups of 4 warps, taking alternate stages
+constexpr int kTcEpiWarp = 2 + 4 * kTcDecGroups;   // first epilogue warp
+constexpr int kTcThreads = 32 * (kTcEpiWarp + 4);  // producer, MMA, decoders, 4 epilogue warps
 constexpr int kTcPStage = kTcRows * 32; // packed bytes per stage: 4 KB
 constexpr int kTcBox = 32;              // output box: 32 tokens x 32 weight rows
+constexpr int kTcEpiBufs = 2;          // 4 KB output staging buffers per epilogue warp
 
 struct GemmTcArgs {
     int64_t M, N, K;
     int nk;                 // k stages: K_pad / 128
+    int tiles_n, tiles_m;   // weight-row tiles (128 rows) and token tiles (BT tokens)
+    int splits;             // K-splits; work units = tiles_n * tiles_m * splits
     int tma_store;          // 1: outputs leave through TMA stores of boxes (y rows 16-byte strided)
     int sps;                // k stages per split (split-K over gridDim.z)
     int reduce;             // 1: add int32 results into the (zeroed) output instead of storing them
@@ -66,26 +77,27 @@ struct GemmTcArgs {
     const float *gamma;     // weight scale (BitLinear)
 };
 
-// Shared-memory plan: SA activation stages (at least 32 KB: the epilogue
-// stages its output boxes there), SP packed stages, mbarriers, the
-// tensor-memory base and the abort flag.  Tensor memory: BT accumulator
-// columns, then SC code stages of 32 columns.
+// Shared-memory plan: SA activation stages, SP packed stages, the epilogue's
+// output boxes (4 warps x kTcEpiBufs x 4 KB), mbarriers, the tensor-memory base and the
+// abort flag.  Tensor memory: two accumulators of BT columns, then SC code
+// stages of 32 columns.
 template <int BT, int SA, int SC, int SP>
 struct TcSmem {
     static constexpr int kAStage = BT * kTcBK;
     static constexpr int kA = 0;
-    static constexpr int kARing = SA * kAStage > 32768 ? SA * kAStage : 32768;
-    static constexpr int kP = kA + kARing;                      // 1024-aligned (multiples of 1 KB above)
-    static constexpr int kBars = kP + SP * kTcPStage;
-    // a_full, a_empty, p_full, p_empty, c_full, c_empty, accum, drain
-    static constexpr int kBarCount = 2 * SA + 2 * SP + 2 * SC + 2;
+    static constexpr int kP = kA + SA * kAStage;                 // 1024-aligned (multiples of 1 KB)
+    static constexpr int kE = kP + SP * kTcPStage;
+    static constexpr int kBars = kE + 4 * kTcEpiBufs * 4096;
+    // a_full, a_empty, p_full, p_empty, c_full, c_empty, accum_full x 2, accum_empty x 2, drain
+    static constexpr int kBarCount = 2 * SA + 2 * SP + 2 * SC + 5;
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kBytes = kMisc + 16;
-    static constexpr int kCodeCol = BT;                          // first code-stage column
-    static constexpr int kTmemNeed = BT + 32 * SC;
+    static constexpr int kCodeCol = 2 * BT;                      // first code-stage column
+    static constexpr int kTmemNeed = 2 * BT + 32 * SC;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "tensor memory");
+    static_assert(kAStage % 1024 == 0, "128-byte swizzled stages are 1024-byte aligned");
 };
 
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
@@ -196,12 +208,25 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Work unit u -> (split, token tile, weight-row tile), weight-row tiles fastest.
+struct TcUnit {
+    int z, mt, nt;
+};
+__device__ __forceinline__ TcUnit tc_unit(const GemmTcArgs &a, int u) {
+    TcUnit t;
+    t.nt = u % a.tiles_n;
+    const int r = u / a.tiles_n;
+    t.mt = r % a.tiles_m;
+    t.z = r / a.tiles_m;
+    return t;
+}
+
 template <int BT, bool BF16_OUT, int SA, int SC, int SP>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
                         const __grid_constant__ CUtensorMap ymap, const GemmTcArgs a) {
     using L = TcSmem<BT, SA, SC, SP>;
-    static_assert(BT == 16 || BT % 32 == 0, "token tile");
+    static_assert(BT % 16 == 0 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBars);
@@ -211,15 +236,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *p_empty = p_full + SP;
     uint64_t *c_full = p_empty + SP;
     uint64_t *c_empty = c_full + SC;
-    uint64_t *accum_full = c_empty + SC;
-    uint64_t *drain = accum_full + 1;
+    uint64_t *accum_full = c_empty + SC;   // [2]
+    uint64_t *accum_empty = accum_full + 2; // [2]
+    uint64_t *drain = accum_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * kTcRows, m0 = (int64_t)blockIdx.y * BT;
-    const int kbase = blockIdx.z * a.sps;  // this split's first k stage
-    const int nk = min(a.sps, a.nk - kbase);
+    const int units = a.tiles_n * a.tiles_m * a.splits;
+    auto unit_stages = [&](const TcUnit &t) { return min(a.sps, a.nk - t.z * a.sps); };
 
     // ---- set-up: descriptors, barriers, tensor memory
     if (threadIdx.x == 0) {
@@ -238,7 +263,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&c_full[s], 4);     // one arrival per decoder warp
             mbar_init(&c_empty[s], 1);    // tcgen05.commit
         }
-        mbar_init(accum_full, 1);
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(&accum_full[d], 1);   // tcgen05.commit
+            mbar_init(&accum_empty[d], 4);  // one arrival per epilogue warp
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -259,142 +287,200 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            int ia = 0, ip = 0;
+            // cursors (unit, stage) of the next activation and packed loads; ia /
+            // ip count the loads issued over all of this CTA's units
+            int ua = blockIdx.x, ka = 0, up = blockIdx.x, kp = 0, ia = 0, ip = 0;
+            TcUnit ta = tc_unit(a, ua), tp = ta;
             auto issue_p = [&]() {
                 mbar_arrive_expect_tx(&p_full[ip % SP], kTcPStage);
-                tma_load_2d(sm + L::kP + (ip % SP) * kTcPStage, &pmap, (kbase + ip) * 32, (int)n0, &p_full[ip % SP]);
+                tma_load_2d(sm + L::kP + (ip % SP) * kTcPStage, &pmap, (tp.z * a.sps + kp) * 32, tp.nt * kTcRows,
+                            &p_full[ip % SP]);
                 ++ip;
+                if (++kp == unit_stages(tp)) {
+                    kp = 0;
+                    up += gridDim.x;
+                    if (up < units) tp = tc_unit(a, up);
+                }
             };
             // weights never depend on an earlier kernel; activations may
-            while (ip < nk && ip < SP) issue_p();
+            while (up < units && ip < SP) issue_p();
             pdl_wait();
-            bool ok = true;
-            while (ok && (ia < nk || ip < nk)) {
-                if (ia < nk && (ia < SA || mbar_try_wait(&a_empty[ia % SA], (uint32_t)((ia / SA) - 1) & 1u))) {
+            // poll both rings without blocking on either (a blocking wait on one
+            // would hold back the other); the idle time is bounded like every wait
+            uint64_t idle_since = 0;
+            while (ua < units || up < units) {
+                bool issued = false;
+                if (ua < units && (ia < SA || mbar_test_wait(&a_empty[ia % SA], (uint32_t)((ia / SA) - 1) & 1u))) {
                     mbar_arrive_expect_tx(&a_full[ia % SA], L::kAStage);
-                    tma_load_2d(sm + L::kA + (ia % SA) * L::kAStage, &amap, (kbase + ia) * kTcBK, (int)m0,
+                    tma_load_2d(sm + L::kA + (ia % SA) * L::kAStage, &amap, (ta.z * a.sps + ka) * kTcBK, ta.mt * BT,
                                 &a_full[ia % SA]);
                     ++ia;
-                    continue;
+                    if (++ka == unit_stages(ta)) {
+                        ka = 0;
+                        ua += gridDim.x;
+                        if (ua < units) ta = tc_unit(a, ua);
+                    }
+                    issued = true;
                 }
-                if (ip < nk && mbar_try_wait(&p_empty[ip % SP], (uint32_t)((ip / SP) - 1) & 1u)) {
+                if (up < units && mbar_test_wait(&p_empty[ip % SP], (uint32_t)((ip / SP) - 1) & 1u)) {
                     issue_p();
+                    issued = true;
+                }
+                if (issued) {
+                    idle_since = 0;
                     continue;
                 }
-                // neither ring has a free stage: wait (bounded) for the one further behind
-                if (ia < nk && (ip >= nk || ia <= ip))
-                    ok = tc_wait(&a_empty[ia % SA], (uint32_t)((ia / SA) - 1) & 1u, abort_flag);
-                else
-                    ok = tc_wait(&p_empty[ip % SP], (uint32_t)((ip / SP) - 1) & 1u, abort_flag);
+                if (*abort_flag) break;
+                const uint64_t now = global_timer_ns();
+                if (idle_since == 0) {
+                    idle_since = now;
+                } else if (now - idle_since > kWaitLimitNs) {
+                    record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                __nanosleep(20);
             }
             // make sure no copy is still landing in shared memory when the CTA leaves
-            for (int kb = ia - SA < 0 ? 0 : ia - SA; kb < ia; ++kb)
-                mbar_wait_bounded(&a_full[kb % SA], (uint32_t)(kb / SA) & 1u);
-            for (int kb = ip - SP < 0 ? 0 : ip - SP; kb < ip; ++kb)
-                mbar_wait_bounded(&p_full[kb % SP], (uint32_t)(kb / SP) & 1u);
+            for (int i = ia - SA < 0 ? 0 : ia - SA; i < ia; ++i)
+                mbar_wait_bounded(&a_full[i % SA], (uint32_t)(i / SA) & 1u);
+            for (int i = ip - SP < 0 ? 0 : ip - SP; i < ip; ++i)
+                mbar_wait_bounded(&p_full[i % SP], (uint32_t)(i / SP) & 1u);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_i8(BT);
             bool ok = true;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int sa = kb % SA, sc = kb % SC;
-                if (!tc_wait(&a_full[sa], (uint32_t)(kb / SA) & 1u, abort_flag) ||
-                    !tc_wait(&c_full[sc], (uint32_t)(kb / SC) & 1u, abort_flag)) {
+            int g = 0;  // stages consumed over all units
+            int li = 0;
+            for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++li) {
+                const int d = li & 1;
+                // the epilogue has drained this accumulator's previous unit
+                if (li >= 2 && !tc_wait(&accum_empty[d], (uint32_t)((li >> 1) - 1) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t bs = smem_u32(sm + L::kA + sa * L::kAStage);
-                const uint32_t ac = tmem + (uint32_t)(L::kCodeCol + 32 * sc);
+                const uint32_t dt = tmem + (uint32_t)(d * BT);
+                const int ns = unit_stages(tc_unit(a, u));
+                for (int kb = 0; kb < ns; ++kb, ++g) {
+                    const int sa = g % SA, sc = g % SC;
+                    if (!tc_wait(&a_full[sa], (uint32_t)(g / SA) & 1u, abort_flag) ||
+                        !tc_wait(&c_full[sc], (uint32_t)(g / SC) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t bs = smem_u32(sm + L::kA + sa * L::kAStage);
+                    const uint32_t ac = tmem + (uint32_t)(L::kCodeCol + 32 * sc);
 #pragma unroll
-                for (int kk = 0; kk < kTcBK / 32; ++kk)
-                    umma_i8_ts(tmem, ac + 8 * kk, umma_desc_sw128(bs + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&a_empty[sa]);
-                umma_commit(&c_empty[sc]);
+                    for (int kk = 0; kk < kTcBK / 32; ++kk)
+                        umma_i8_ts(dt, ac + 8 * kk, umma_desc_sw128(bs + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&a_empty[sa]);
+                    umma_commit(&c_empty[sc]);
+                }
+                if (ok) umma_commit(&accum_full[d]);
             }
-            if (ok) {
-                umma_commit(accum_full);
-            } else {
+            if (!ok) {
                 // drain the MMAs already issued before tensor memory is released
                 umma_commit(drain);
                 mbar_wait_bounded(drain, 0);
             }
         }
-    } else {
-        // ---------------------------------------------------------------- decoders, then epilogue
+    } else if (warp < kTcEpiWarp) {
+        // ---------------------------------------------------------------- decoders
         const int quarter = warp & 3;            // tensor-memory lanes 32 * quarter ...
-        const int row = quarter * 32 + lane;     // this thread's weight row in the tile
+        const int group = (warp - 2) >> 2;       // stages g with g % kTcDecGroups == group
+        const int row = quarter * 32 + lane;     // this thread's weight row in a tile
         const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
+        const int sw = (row >> 2) & 1;
+        int g = 0;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % SC, ps = kb % SP;
-            // the packed tile has landed and the MMAs that last read this code stage are done
-            if (!tc_wait(&p_full[ps], (uint32_t)(kb / SP) & 1u, abort_flag) ||
-                (kb >= SC && !tc_wait(&c_empty[s], (uint32_t)((kb / SC) - 1) & 1u, abort_flag))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // the packed tile arrives with the 32-byte swizzle: 16-byte half h of
-            // row r sits at r * 32 + ((h ^ ((r >> 2) & 1)) * 16)
-            const uint8_t *pr = sm + L::kP + ps * kTcPStage + row * 32;
-            const int sw = (row >> 2) & 1;
-            const uint4 p0 = *reinterpret_cast<const uint4 *>(pr + (sw << 4));
-            const uint4 p1 = *reinterpret_cast<const uint4 *>(pr + ((sw ^ 1) << 4));
-            const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            uint32_t c[32];
+        for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+            const int ns = unit_stages(tc_unit(a, u));
+            for (int kb = 0; kb < ns; ++kb, ++g) {
+                if (g % kTcDecGroups != group) continue;
+                const int s = g % SC, ps = g % SP;
+                // the packed tile has landed and the MMAs that last read this code stage are done
+                if (!tc_wait(&p_full[ps], (uint32_t)(g / SP) & 1u, abort_flag) ||
+                    (g >= SC && !tc_wait(&c_empty[s], (uint32_t)((g / SC) - 1) & 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // the packed tile arrives with the 32-byte swizzle: 16-byte half h of
+                // row r sits at r * 32 + ((h ^ ((r >> 2) & 1)) * 16)
+                const uint8_t *pr = sm + L::kP + ps * kTcPStage + row * 32;
+                const uint4 p0 = *reinterpret_cast<const uint4 *>(pr + (sw << 4));
+                const uint4 p1 = *reinterpret_cast<const uint4 *>(pr + ((sw ^ 1) << 4));
+                const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                uint32_t c[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 8; ++i) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) c[4 * i + j] = (((w[i] >> (2 * j)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                    for (int j = 0; j < 4; ++j)
+                        c[4 * i + j] = (((w[i] >> (2 * j)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                }
+                __syncwarp();  // every lane has its packed row in registers
+                if (lane == 0)
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&p_empty[ps])) : "memory");
+                tmem_st32(tq + (uint32_t)(L::kCodeCol + 32 * s), c);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&c_full[s])) : "memory");
             }
-            __syncwarp();  // every lane has its packed row in registers
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&p_empty[ps])) : "memory");
-            tmem_st32(tq + (uint32_t)(L::kCodeCol + 32 * s), c);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&c_full[s])) : "memory");
         }
-        // epilogue: thread (quarter, lane) owns accumulator lane `row`, one
-        // column per token of the tile
-        if (ok && tc_wait(accum_full, 0, abort_flag)) {
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint8_t *wbuf = sm + L::kE + quarter * kTcEpiBufs * 4096;
+        constexpr int kTok = BT < kTcBox ? BT : kTcBox;
+        bool waited_pdl = false;
+        int nbox = 0;  // boxes this warp has stored (its staging buffers take turns)
+        int li = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++li) {
+            const int d = li & 1;
+            if (!tc_wait(&accum_full[d], (uint32_t)(li >> 1) & 1u, abort_flag)) break;
             tc_fence_after();
+            if (!waited_pdl) {
+                pdl_wait();  // the outputs may still be read by the previous kernel
+                waited_pdl = true;
+            }
+            const TcUnit t = tc_unit(a, u);
+            const int64_t n0 = (int64_t)t.nt * kTcRows, m0 = (int64_t)t.mt * BT;
             const int64_t n = n0 + row;
+            const uint32_t dt = tq + (uint32_t)(d * BT);
             // BitLinear factor gamma / s_m of token c0 + lane (lanes share it by shuffle)
             auto token_factor = [&](int c0) {
                 const int64_t m = m0 + c0 + lane;
                 return (BF16_OUT && m < a.M) ? __fdiv_rn(*a.gamma, a.s_act[m]) : 0.0f;
             };
-            pdl_wait();  // the outputs may still be read by the previous kernel
             uint32_t v[16];
             if (a.tma_store) {
-                // boxes of (up to) 32 tokens x 32 weight rows, row-major by token
-                // as y is; two 4 KB buffers per warp in the freed activation ring
-                uint8_t *wbuf = sm + L::kA + quarter * 2 * 4096;
-                constexpr int kTok = BT < kTcBox ? BT : kTcBox;
+                // boxes of (up to) 32 tokens x 32 weight rows, row-major by token as y is
 #pragma unroll 1
-                for (int c0 = 0, it = 0; c0 < BT; c0 += kTok, ++it) {
-                    uint8_t *buf = wbuf + (it & 1) * 4096;
-                    if (it >= 2) {
-                        if (lane == 0) tma_store_wait_read<1>();
+                for (int c0 = 0; c0 < BT; c0 += kTok, ++nbox) {
+                    uint8_t *buf = wbuf + (nbox % kTcEpiBufs) * 4096;
+                    if (nbox >= kTcEpiBufs) {
+                        if (lane == 0) tma_store_wait_read<kTcEpiBufs - 1>();
                         __syncwarp();
                     }
                     const float fl = token_factor(c0);
 #pragma unroll
                     for (int h = 0; h < kTok / 16; ++h) {
-                        tmem_ld16(tq + (uint32_t)(c0 + 16 * h), v);
+                        tmem_ld16(dt + (uint32_t)(c0 + 16 * h), v);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const int t = 16 * h + i;
+                            const int tk = 16 * h + i;
                             if (BF16_OUT)
-                                reinterpret_cast<uint16_t *>(buf)[t * 32 + lane] = float_to_bf16_bits_rn(
-                                    __fmul_rn((float)(int)v[i], __shfl_sync(0xffffffffu, fl, t)));
+                                reinterpret_cast<uint16_t *>(buf)[tk * 32 + lane] = float_to_bf16_bits_rn(
+                                    __fmul_rn((float)(int)v[i], __shfl_sync(0xffffffffu, fl, tk)));
                             else
-                                reinterpret_cast<uint32_t *>(buf)[t * 32 + lane] = v[i];
+                                reinterpret_cast<uint32_t *>(buf)[tk * 32 + lane] = v[i];
                         }
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -406,12 +492,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             tma_store_2d(&ymap, (int)(n0 + quarter * 32), (int)(m0 + c0), buf);
                     }
                 }
-                if (lane == 0) tma_store_wait_all();
-                __syncwarp();
             } else {
 #pragma unroll 1
                 for (int c0 = 0; c0 < BT; c0 += 16) {
-                    tmem_ld16(tq + (uint32_t)c0, v);
+                    tmem_ld16(dt + (uint32_t)c0, v);
                     const float fl = token_factor(c0);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -428,7 +512,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
             }
+            // every accumulator load of this unit is complete: release the accumulator
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty[d])) : "memory");
         }
+        if (lane == 0) tma_store_wait_all();
+        __syncwarp();
     }
 
     // ---- teardown: every tensor-memory access is complete before the free

@@ -3,7 +3,8 @@
 Ragged shapes (M, N not multiples of the tile, K not a multiple of the
 128-byte stage or of 16, which makes the library repack the activations), every
 token-tile width with and without a K-split (forced in child processes through
-BITNET_GEMV_TUNE, read once per process), int32 and BitLinear bf16 outputs.
+BITNET_GEMV_TUNE, read once per process), problems with many work units per
+persistent CTA, int32 and BitLinear bf16 outputs.
 """
 import json
 import os
@@ -75,7 +76,8 @@ import oracle
 import ternary_weight_bit_w2a8_b200 as bn
 from ternary_weight_bit_w2a8_b200 import synth
 out = {}
-for (M, N, K) in [(130, 300, 1000), (256, 520, 2560), (9, 1000, 384), (40, 129, 640), (300, 64, 4096)]:
+for (M, N, K) in [(130, 300, 1000), (256, 520, 2560), (9, 1000, 384), (40, 129, 640), (300, 64, 4096),
+                  (2000, 4096, 256)]:
     q, w = synth.uniform_int8_ternary(N, K, seed=M * N + K, M=M)
     q[-1, :] = -128
     y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()), N)
@@ -96,7 +98,9 @@ print(json.dumps(out))
 """
 
 
-# token tile 1..5 = 256, 128, 64, 32, 16 tokens; S = K-splits (0: none when a tile is forced)
+# token tile 1..5 = 192, 128, 64, 32, 16 tokens; S = K-splits (0: none when a tile is forced).  The
+# 2000 x 4096 problem gives every persistent CTA several work units, so both
+# accumulators are reused many times.
 @pytest.mark.parametrize("tile,S", [(1, 0), (2, 0), (3, 0), (4, 0), (5, 0), (1, 3), (3, 5), (5, 2)])
 def test_tc_every_tile_width(tile, S):
     env = dict(os.environ)
