@@ -455,20 +455,20 @@ constexpr int kTcNumBT = 5;
 constexpr int kTcBTs[kTcNumBT] = {192, 128, 64, 32, 16};
 using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
-// Rings (activation, code, packed stages) per token-tile width.  The 192- and
-// 128-token variants take all 512 tensor-memory columns (2 accumulators + 4
-// code stages) and more than half an SM's shared memory, so one CTA per SM;
-// the narrower ones take 256 columns and at most two CTAs share an SM.
+// Rings (activation, code, packed stages of 256 k) per token-tile width.  The
+// 192-, 128- and 64-token variants take all 512 tensor-memory columns (2
+// accumulators + code stages of 64 columns) and more than half an SM's shared
+// memory, so one CTA per SM; the narrower ones take 256 columns.
 TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
     static const TcKernel k[2 * kTcNumBT] = {
-        gemm_w2a8_tc_kernel<192, false, 4, 4, 6>, gemm_w2a8_tc_kernel<128, false, 5, 4, 6>,
-        gemm_w2a8_tc_kernel<64, false, 6, 4, 6>,  gemm_w2a8_tc_kernel<32, false, 8, 4, 8>,
-        gemm_w2a8_tc_kernel<16, false, 8, 4, 8>,  gemm_w2a8_tc_kernel<192, true, 4, 4, 6>,
-        gemm_w2a8_tc_kernel<128, true, 5, 4, 6>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
-        gemm_w2a8_tc_kernel<32, true, 8, 4, 8>,   gemm_w2a8_tc_kernel<16, true, 8, 4, 8>};
-    static const size_t raw[kTcNumBT] = {TcSmem<192, 4, 4, 6>::kBytes, TcSmem<128, 5, 4, 6>::kBytes,
-                                         TcSmem<64, 6, 4, 6>::kBytes, TcSmem<32, 8, 4, 8>::kBytes,
-                                         TcSmem<16, 8, 4, 8>::kBytes};
+        gemm_w2a8_tc_kernel<192, false, 3, 2, 4>, gemm_w2a8_tc_kernel<128, false, 4, 4, 4>,
+        gemm_w2a8_tc_kernel<64, false, 6, 4, 6>,  gemm_w2a8_tc_kernel<32, false, 8, 3, 6>,
+        gemm_w2a8_tc_kernel<16, false, 8, 3, 6>,  gemm_w2a8_tc_kernel<192, true, 3, 2, 4>,
+        gemm_w2a8_tc_kernel<128, true, 4, 4, 4>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
+        gemm_w2a8_tc_kernel<32, true, 8, 3, 6>,   gemm_w2a8_tc_kernel<16, true, 8, 3, 6>};
+    static const size_t raw[kTcNumBT] = {TcSmem<192, 3, 2, 4>::kBytes, TcSmem<128, 4, 4, 4>::kBytes,
+                                         TcSmem<64, 6, 4, 6>::kBytes, TcSmem<32, 8, 3, 6>::kBytes,
+                                         TcSmem<16, 8, 3, 6>::kBytes};
     *smem = raw[bt_idx] + 1024;  // + alignment slack
     return k[(bf16 ? kTcNumBT : 0) + bt_idx];
 }
@@ -493,7 +493,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
     TcPlan p{};
     const GemvTune &tn = gemv_tune();
-    const int nk = (int)(k_pad(K) / kTcBK);
+    const int nk = (int)ceil_div(k_pad(K), kTcSK);
     const int64_t nt = ceil_div(N, kTcRows);
     int first = kTcNumBT - 1;
     while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else the widest
@@ -501,7 +501,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     for (int i = first; i < kTcNumBT; ++i) {
         const int BT = kTcBTs[i];
         const int64_t tiles = nt * ceil_div(M, BT);
-        const double stage_us = std::max(0.41 * BT / 256.0, 0.40);
+        const double stage_us = std::max(0.82 * BT / 256.0, 0.45);  // a stage of 256 k
         const double out_us = (double)M * (double)N * 4.0 / 1.4e6;  // one pass over the int32 output
         for (int S = 1; S <= 16 && S <= nk; ++S) {
             if (S > 1 && tiles >= kRefSMs) break;
@@ -564,10 +564,10 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         const int64_t row_bytes = packed_row_bytes(K);
         const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
         const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-        const cuuint32_t box[2] = {32u, (cuuint32_t)kTcRows};
+        const cuuint32_t box[2] = {(cuuint32_t)kTcPRow, (cuuint32_t)kTcRows};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
-                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITNET_ERR_CUDA;
     }
@@ -594,7 +594,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.M = M;
     a.N = N;
     a.K = K;
-    a.nk = (int)(k_pad(K) / kTcBK);
+    a.nk = (int)ceil_div(k_pad(K), kTcSK);
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.s_act = s_act;

@@ -10,25 +10,27 @@
 // kernel is persistent, one CTA per SM looping over work units.
 //   - Work unit: 128 weight rows (UMMA M) x BT tokens (UMMA N) x one K-split;
 //     units are dealt round-robin to the CTAs, weight-row tiles fastest.  A
-//     unit is done in stages of 128 k; its accumulator D[n, m] takes 128 TMEM
+//     unit is done in stages of 256 k (8 MMAs per hand-over between decoders
+//     and tensor core: on B200 the hand-overs, not the MMAs, bounded the stage
+//     rate at 128 k per stage); its accumulator D[n, m] takes 128 TMEM
 //     lanes x BT columns, and two accumulators alternate so that one unit's
 //     epilogue overlaps the next unit's main loop.
 //   - Warp 0, one lane: TMA producer of two rings that run on across units,
-//     each with full / empty mbarriers: activation tiles (int8 [BT tokens x
-//     128 bytes], 128-byte swizzle: the canonical K-major B operand; SA stages)
-//     and packed weight tiles (layout v1, [128 rows x 32 bytes], 32-byte
-//     swizzle; SP stages).  The first packed tiles are requested before
+//     each with full / empty mbarriers: activation tiles (two int8 boxes of
+//     [BT tokens x 128 bytes], 128-byte swizzle: the canonical K-major B
+//     operand; SA stages) and packed weight tiles (layout v1, [128 rows x 64
+//     bytes], 64-byte swizzle; SP stages).  The first packed tiles are requested before
 //     griddepcontrol.wait (weights never depend on an earlier kernel).
 //   - Warps 2..9: decoders, two groups of four that take alternate stages (a
 //     group's tensor-memory store latency hides behind the other group's
 //     work).  A thread owns one weight row (its warp's TMEM lane quarter).
-//     Per stage the row's 8 packed words (128 k) become 32 words of
+//     Per stage the row's 16 packed words (256 k) become 64 words of
 //     signed codes: (word >> 2j) & 0x03030303 gives the codes c of 4
 //     consecutive k, and ((c + 0x7F7F7F7F) ^ 0x80808080) is c - 1 in every
-//     byte with no carry between bytes.  One tcgen05.st writes the 32 words
-//     into a code stage of tensor memory (SC stages of 32 columns).
-//   - Warp 1: allocates tensor memory and, from one lane, issues per stage four
-//     K = 32 MMAs (A = codes in tensor memory, B = activations in shared
+//     byte with no carry between bytes.  Two tcgen05.st write the 64 words
+//     into a code stage of tensor memory (SC stages of 64 columns).
+//   - Warp 1: allocates tensor memory and, from one lane, issues per stage
+//     eight K = 32 MMAs (A = codes in tensor memory, B = activations in shared
 //     memory, s8 x s8 -> s32) into the unit's accumulator; tcgen05.commit on
 //     per-stage mbarriers releases the activation and code stages, and on a
 //     per-accumulator mbarrier hands a finished unit to the epilogue.
@@ -55,11 +57,13 @@
 namespace bitnet {
 
 constexpr int kTcRows = 128;            // weight rows per tile (UMMA M)
-constexpr int kTcBK = 128;              // k per stage (bytes of an activation row)
+constexpr int kTcBK = 128;              // k per activation box (bytes of a 128-byte swizzled row)
+constexpr int kTcSK = 256;              // k per stage: two activation boxes, 8 MMAs of K = 32
+constexpr int kTcPRow = kTcSK / 4;      // packed bytes of one weight row per stage: 64
 constexpr int kTcDecGroups = 2;        // decoder groups of 4 warps, taking alternate stages
 constexpr int kTcEpiWarp = 2 + 4 * kTcDecGroups;   // first epilogue warp
 constexpr int kTcThreads = 32 * (kTcEpiWarp + 4);  // producer, MMA, decoders, 4 epilogue warps
-constexpr int kTcPStage = kTcRows * 32; // packed bytes per stage: 4 KB
+constexpr int kTcPStage = kTcRows * kTcPRow;  // packed bytes per stage: 8 KB
 constexpr int kTcBox = 32;              // output box: 32 tokens x 32 weight rows
 constexpr int kTcEpiBufs = 2;          // 4 KB output staging buffers per epilogue warp
 
@@ -80,10 +84,11 @@ struct GemmTcArgs {
 // Shared-memory plan: SA activation stages, SP packed stages, the epilogue's
 // output boxes (4 warps x kTcEpiBufs x 4 KB), mbarriers, the tensor-memory base and the
 // abort flag.  Tensor memory: two accumulators of BT columns, then SC code
-// stages of 32 columns.
+// stages of 64 columns (256 k).
 template <int BT, int SA, int SC, int SP>
 struct TcSmem {
-    static constexpr int kAStage = BT * kTcBK;
+    static constexpr int kAHalf = BT * kTcBK;                    // one activation box
+    static constexpr int kAStage = 2 * kAHalf;
     static constexpr int kA = 0;
     static constexpr int kP = kA + SA * kAStage;                 // 1024-aligned (multiples of 1 KB)
     static constexpr int kE = kP + SP * kTcPStage;
@@ -93,11 +98,12 @@ struct TcSmem {
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kCodeCol = 2 * BT;                      // first code-stage column
-    static constexpr int kTmemNeed = 2 * BT + 32 * SC;
+    static constexpr int kCodeCols = kTcSK / 4;                  // 32-bit columns of one code stage
+    static constexpr int kTmemNeed = 2 * BT + kCodeCols * SC;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "tensor memory");
-    static_assert(kAStage % 1024 == 0, "128-byte swizzled stages are 1024-byte aligned");
+    static_assert(kAHalf % 1024 == 0, "128-byte swizzled boxes are 1024-byte aligned");
 };
 
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
@@ -147,9 +153,9 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Writes 32 consecutive 32-bit columns of this thread's tensor-memory lane and
-// waits until the writes are done.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+// Writes 32 consecutive 32-bit columns of this thread's tensor-memory lane
+// (tcgen05.wait::st, below, waits until such writes are done).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
         "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
@@ -158,8 +164,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
         "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Bounded wait that also gives up when another role has raised the abort flag.
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
@@ -293,7 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             TcUnit ta = tc_unit(a, ua), tp = ta;
             auto issue_p = [&]() {
                 mbar_arrive_expect_tx(&p_full[ip % SP], kTcPStage);
-                tma_load_2d(sm + L::kP + (ip % SP) * kTcPStage, &pmap, (tp.z * a.sps + kp) * 32, tp.nt * kTcRows,
+                tma_load_2d(sm + L::kP + (ip % SP) * kTcPStage, &pmap, (tp.z * a.sps + kp) * kTcPRow, tp.nt * kTcRows,
                             &p_full[ip % SP]);
                 ++ip;
                 if (++kp == unit_stages(tp)) {
@@ -312,8 +319,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bool issued = false;
                 if (ua < units && (ia < SA || mbar_test_wait(&a_empty[ia % SA], (uint32_t)((ia / SA) - 1) & 1u))) {
                     mbar_arrive_expect_tx(&a_full[ia % SA], L::kAStage);
-                    tma_load_2d(sm + L::kA + (ia % SA) * L::kAStage, &amap, (ta.z * a.sps + ka) * kTcBK, ta.mt * BT,
-                                &a_full[ia % SA]);
+                    const int kx = (ta.z * a.sps + ka) * kTcSK;
+                    uint8_t *ad = sm + L::kA + (ia % SA) * L::kAStage;
+                    tma_load_2d(ad, &amap, kx, ta.mt * BT, &a_full[ia % SA]);
+                    tma_load_2d(ad + L::kAHalf, &amap, kx + kTcBK, ta.mt * BT, &a_full[ia % SA]);
                     ++ia;
                     if (++ka == unit_stages(ta)) {
                         ka = 0;
@@ -373,10 +382,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t bs = smem_u32(sm + L::kA + sa * L::kAStage);
-                    const uint32_t ac = tmem + (uint32_t)(L::kCodeCol + 32 * sc);
+                    const uint32_t ac = tmem + (uint32_t)(L::kCodeCol + L::kCodeCols * sc);
 #pragma unroll
-                    for (int kk = 0; kk < kTcBK / 32; ++kk)
-                        umma_i8_ts(dt, ac + 8 * kk, umma_desc_sw128(bs + kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kTcSK / 32; ++kk)
+                        umma_i8_ts(dt, ac + 8 * kk,
+                                   umma_desc_sw128(bs + (kk >> 2) * L::kAHalf + (kk & 3) * 32), idesc,
+                                   (kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&a_empty[sa]);
                     umma_commit(&c_empty[sc]);
                 }
@@ -394,7 +405,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int group = (warp - 2) >> 2;       // stages g with g % kTcDecGroups == group
         const int row = quarter * 32 + lane;     // this thread's weight row in a tile
         const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
-        const int sw = (row >> 2) & 1;
+        const int sw = (row >> 1) & 3;
         int g = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
@@ -409,15 +420,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                // the packed tile arrives with the 32-byte swizzle: 16-byte half h of
-                // row r sits at r * 32 + ((h ^ ((r >> 2) & 1)) * 16)
-                const uint8_t *pr = sm + L::kP + ps * kTcPStage + row * 32;
-                const uint4 p0 = *reinterpret_cast<const uint4 *>(pr + (sw << 4));
-                const uint4 p1 = *reinterpret_cast<const uint4 *>(pr + ((sw ^ 1) << 4));
-                const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                uint32_t c[32];
+                // the packed tile arrives with the 64-byte swizzle: 16-byte chunk c
+                // of row r sits at r * 64 + ((c ^ ((r >> 1) & 3)) * 16)
+                const uint8_t *pr = sm + L::kP + ps * kTcPStage + row * kTcPRow;
+                uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint4 p = *reinterpret_cast<const uint4 *>(pr + ((ch ^ sw) << 4));
+                    w[4 * ch] = p.x;
+                    w[4 * ch + 1] = p.y;
+                    w[4 * ch + 2] = p.z;
+                    w[4 * ch + 3] = p.w;
+                }
+                uint32_t c[64];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         c[4 * i + j] = (((w[i] >> (2 * j)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
@@ -425,7 +442,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 __syncwarp();  // every lane has its packed row in registers
                 if (lane == 0)
                     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&p_empty[ps])) : "memory");
-                tmem_st32(tq + (uint32_t)(L::kCodeCol + 32 * s), c);
+                const uint32_t cs = tq + (uint32_t)(L::kCodeCol + L::kCodeCols * s);
+                tmem_st32(cs, c);
+                tmem_st32(cs + 32, c + 32);
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
