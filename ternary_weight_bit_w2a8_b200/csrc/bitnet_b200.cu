@@ -476,9 +476,9 @@ TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
 // Token-tile width and K-split of the tensor-core GEMM, from a small cost
 // model of the persistent kernel on the B200's 148 SMs (so the workspace a
 // shape needs is fixed whatever the device): an SM runs its work units one
-// after another; a stage of 128 k took about 0.4 us for every token-tile
+// after another; a stage of 256 k took about 0.6 us for every token-tile
 // width measured on B200 (the hand-over between decoders and tensor core
-// bounds it, not the MMA), so the model charges max(0.4 us, the MMA time);
+// bounds it, not the MMA), so the model charges max(0.6 us, the MMA time);
 // the pipeline fill and the last epilogue add ~2 us.  A K-split is considered
 // only when the tiles do not fill the SMs; it adds a launch (~2.5 us) plus
 // the zeroing of the int32 output and one reduce-add pass over it per split,
@@ -501,7 +501,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     for (int i = first; i < kTcNumBT; ++i) {
         const int BT = kTcBTs[i];
         const int64_t tiles = nt * ceil_div(M, BT);
-        const double stage_us = std::max(0.82 * BT / 256.0, 0.45);  // a stage of 256 k
+        const double stage_us = std::max(0.82 * BT / 256.0, 0.60);  // a stage of 256 k
         const double out_us = (double)M * (double)N * 4.0 / 1.4e6;  // one pass over the int32 output
         for (int S = 1; S <= 16 && S <= nk; ++S) {
             if (S > 1 && tiles >= kRefSMs) break;
