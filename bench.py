@@ -550,16 +550,28 @@ def run_reference(args):
 
 
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "traffic_gemv_tma_sweep.md")
-TRAFFIC_SOURCES = ("common.cuh", "gemv_tma.cuh", "bitnet_b200.cu")
+TRAFFIC_SOURCES = ("common.cuh", "quant.cuh", "gemv.cuh", "gemv_tma.cuh")
+# the tensor-core GEMM's section of the translation unit (not part of the GEMV)
+TC_SECTION = ("// ------------------------------------------------------------------ tcgen05 GEMM (M > 1)",
+              "// ------------------------------------------------------------------ dispatch")
 
 
 def kernel_source_hash():
-    """sha256 over the sources that decide the GEMV kernel and its launch."""
+    """sha256 over the sources that decide the GEMV kernel and its launch: its
+    headers and the translation unit without the tensor-core GEMM's section."""
     import hashlib
     h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ternary_weight_bit_w2a8_b200", "csrc")
     for name in TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, "ternary_weight_bit_w2a8_b200", "csrc", name), "rb") as f:
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(csrc, "bitnet_b200.cu"), encoding="utf-8") as f:
+        tu = f.read()
+    a = tu.find(TC_SECTION[0])
+    b = tu.find(TC_SECTION[1], a + 1) if a >= 0 else -1
+    if a >= 0 and b > a:
+        tu = tu[:a] + tu[b:]
+    h.update(tu.encode("utf-8"))
     return h.hexdigest()
 
 

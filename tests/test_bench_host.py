@@ -112,3 +112,21 @@ def test_replay_steps_runs_exactly_n_steps():
         steps = [c for t in log for c in t]
         assert len(steps) == n
         assert steps == [i % 7 for i in range(n)]  # every step on the next rotation copy
+
+
+def test_traffic_hash_covers_the_gemv_not_the_tensor_core_gemm(tmp_path, monkeypatch):
+    import shutil
+    src = os.path.join(ROOT, "ternary_weight_bit_w2a8_b200", "csrc")
+    dst = tmp_path / "ternary_weight_bit_w2a8_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    assert h0 == bench.kernel_source_hash()
+    tu = (dst / "bitnet_b200.cu").read_text(encoding="utf-8")
+    a = tu.index(bench.TC_SECTION[0])
+    (dst / "bitnet_b200.cu").write_text(tu[:a + len(bench.TC_SECTION[0])] + "\n// edit\n" +
+                                        tu[a + len(bench.TC_SECTION[0]):], encoding="utf-8")
+    assert bench.kernel_source_hash() == h0          # a tensor-core GEMM edit keeps the GEMV figure
+    (dst / "gemv_tma.cuh").write_text((dst / "gemv_tma.cuh").read_text(encoding="utf-8") + "\n// edit\n",
+                                      encoding="utf-8")
+    assert bench.kernel_source_hash() != h0          # a GEMV edit invalidates it
