@@ -453,22 +453,29 @@ int noalloc_scratch(void **out) {
 // Token-tile widths (UMMA N) of the persistent tensor-core GEMM.
 constexpr int kTcNumBT = 5;
 constexpr int kTcBTs[kTcNumBT] = {192, 128, 64, 32, 16};
+// k per stage of each variant (its packed rows are k / 4 bytes, 64-byte or
+// 128-byte swizzled; its code stages k / 4 tensor-memory columns)
+constexpr int kTcSKs[kTcNumBT] = {256, 512, 256, 256, 256};
+// Time of one stage of each variant with every SM busy, measured on B200 (us):
+// the MMA time for the wide tiles, the decoder-to-tensor-core hand-over
+// (~0.6 us) for the narrow ones.
+constexpr double kTcStageUs[kTcNumBT] = {0.69, 1.12, 0.60, 0.60, 0.60};
 using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
-// Rings (activation, code, packed stages of 256 k) per token-tile width.  The
-// 192-, 128- and 64-token variants take all 512 tensor-memory columns (2
-// accumulators + code stages of 64 columns) and more than half an SM's shared
-// memory, so one CTA per SM; the narrower ones take 256 columns.
+// Rings (activation, code, packed stages) per token-tile width.  The 192-,
+// 128- and 64-token variants take all 512 tensor-memory columns (2
+// accumulators + code stages) and more than half an SM's shared memory, so
+// one CTA per SM; the narrower ones take 256 columns.
 TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
     static const TcKernel k[2 * kTcNumBT] = {
-        gemm_w2a8_tc_kernel<192, false, 3, 2, 4>, gemm_w2a8_tc_kernel<128, false, 4, 4, 4>,
-        gemm_w2a8_tc_kernel<64, false, 6, 4, 6>,  gemm_w2a8_tc_kernel<32, false, 8, 3, 6>,
-        gemm_w2a8_tc_kernel<16, false, 8, 3, 6>,  gemm_w2a8_tc_kernel<192, true, 3, 2, 4>,
-        gemm_w2a8_tc_kernel<128, true, 4, 4, 4>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6>,
-        gemm_w2a8_tc_kernel<32, true, 8, 3, 6>,   gemm_w2a8_tc_kernel<16, true, 8, 3, 6>};
-    static const size_t raw[kTcNumBT] = {TcSmem<192, 3, 2, 4>::kBytes, TcSmem<128, 4, 4, 4>::kBytes,
-                                         TcSmem<64, 6, 4, 6>::kBytes, TcSmem<32, 8, 3, 6>::kBytes,
-                                         TcSmem<16, 8, 3, 6>::kBytes};
+        gemm_w2a8_tc_kernel<192, false, 3, 2, 4, 256>, gemm_w2a8_tc_kernel<128, false, 2, 2, 3, 512>,
+        gemm_w2a8_tc_kernel<64, false, 6, 4, 6, 256>,  gemm_w2a8_tc_kernel<32, false, 8, 3, 6, 256>,
+        gemm_w2a8_tc_kernel<16, false, 8, 3, 6, 256>,  gemm_w2a8_tc_kernel<192, true, 3, 2, 4, 256>,
+        gemm_w2a8_tc_kernel<128, true, 2, 2, 3, 512>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6, 256>,
+        gemm_w2a8_tc_kernel<32, true, 8, 3, 6, 256>,   gemm_w2a8_tc_kernel<16, true, 8, 3, 6, 256>};
+    static const size_t raw[kTcNumBT] = {TcSmem<192, 3, 2, 4, 256>::kBytes, TcSmem<128, 2, 2, 3, 512>::kBytes,
+                                         TcSmem<64, 6, 4, 6, 256>::kBytes, TcSmem<32, 8, 3, 6, 256>::kBytes,
+                                         TcSmem<16, 8, 3, 6, 256>::kBytes};
     *smem = raw[bt_idx] + 1024;  // + alignment slack
     return k[(bf16 ? kTcNumBT : 0) + bt_idx];
 }
@@ -476,15 +483,15 @@ TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
 // Token-tile width and K-split of the tensor-core GEMM, from a small cost
 // model of the persistent kernel on the B200's 148 SMs (so the workspace a
 // shape needs is fixed whatever the device): an SM runs its work units one
-// after another; a stage of 256 k took about 0.6 us for every token-tile
-// width measured on B200 (the hand-over between decoders and tensor core
-// bounds it, not the MMA), so the model charges max(0.6 us, the MMA time);
-// the pipeline fill and the last epilogue add ~2 us.  A K-split is considered
-// only when the tiles do not fill the SMs; it adds a launch (~2.5 us) plus
-// the zeroing of the int32 output and one reduce-add pass over it per split,
-// each at ~1.4 TB/s (measured: a 2-way split of M = 2048, N = 13824 cost more
-// than the whole unsplit GEMM).  Candidates: token tiles from the smallest
-// that holds M (at most 192) down to 16, splits 1..16.
+// after another, each stage taking the variant's measured time (kTcStageUs;
+// at 128 k per stage every variant took ~0.4 us, bounded by the hand-over
+// between decoders and tensor core, which is why the stages are now 256 or
+// 512 k); the pipeline fill and the last epilogue add ~2 us.  A K-split is
+// considered only when the tiles do not fill the SMs; it adds a launch
+// (~2.5 us) plus the zeroing of the int32 output and one reduce-add pass over
+// it per split, each at ~1.4 TB/s (measured: a 2-way split of M = 2048,
+// N = 13824 cost more than the whole unsplit GEMM).  Candidates: token tiles
+// from the smallest that holds M (at most 192) down to 16, splits 1..16.
 struct TcPlan {
     int bt_idx, S, sps;
 };
@@ -493,15 +500,15 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
     TcPlan p{};
     const GemvTune &tn = gemv_tune();
-    const int nk = (int)ceil_div(k_pad(K), kTcSK);
     const int64_t nt = ceil_div(N, kTcRows);
     int first = kTcNumBT - 1;
     while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else the widest
     double best = 1e30;
     for (int i = first; i < kTcNumBT; ++i) {
         const int BT = kTcBTs[i];
+        const int nk = (int)ceil_div(k_pad(K), kTcSKs[i]);
         const int64_t tiles = nt * ceil_div(M, BT);
-        const double stage_us = std::max(0.82 * BT / 256.0, 0.60);  // a stage of 256 k
+        const double stage_us = kTcStageUs[i];
         const double out_us = (double)M * (double)N * 4.0 / 1.4e6;  // one pass over the int32 output
         for (int S = 1; S <= 16 && S <= nk; ++S) {
             if (S > 1 && tiles >= kRefSMs) break;
@@ -519,6 +526,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     }
     // tuning overrides: R = -1..-5 picks the token tile, S the split count
     if (tn.R < 0 && -tn.R <= kTcNumBT) p.bt_idx = -tn.R - 1;
+    const int nk = (int)ceil_div(k_pad(K), kTcSKs[p.bt_idx]);
     if (tn.S > 0) {
         const int S = tn.S < nk ? tn.S : nk;
         p.sps = (int)ceil_div(nk, S);
@@ -564,10 +572,11 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         const int64_t row_bytes = packed_row_bytes(K);
         const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
         const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-        const cuuint32_t box[2] = {(cuuint32_t)kTcPRow, (cuuint32_t)kTcRows};
+        const cuuint32_t box[2] = {(cuuint32_t)(kTcSKs[bi] / 4), (cuuint32_t)kTcRows};
         const cuuint32_t es[2] = {1, 1};
         if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
-                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 kTcSKs[bi] == 512 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITNET_ERR_CUDA;
     }
@@ -594,7 +603,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.M = M;
     a.N = N;
     a.K = K;
-    a.nk = (int)ceil_div(k_pad(K), kTcSK);
+    a.nk = (int)ceil_div(k_pad(K), kTcSKs[bi]);
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.s_act = s_act;

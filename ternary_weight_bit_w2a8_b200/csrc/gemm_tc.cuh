@@ -58,12 +58,9 @@ namespace bitnet {
 
 constexpr int kTcRows = 128;            // weight rows per tile (UMMA M)
 constexpr int kTcBK = 128;              // k per activation box (bytes of a 128-byte swizzled row)
-constexpr int kTcSK = 256;              // k per stage: two activation boxes, 8 MMAs of K = 32
-constexpr int kTcPRow = kTcSK / 4;      // packed bytes of one weight row per stage: 64
 constexpr int kTcDecGroups = 2;        // decoder groups of 4 warps, taking alternate stages
 constexpr int kTcEpiWarp = 2 + 4 * kTcDecGroups;   // first epilogue warp
 constexpr int kTcThreads = 32 * (kTcEpiWarp + 4);  // producer, MMA, decoders, 4 epilogue warps
-constexpr int kTcPStage = kTcRows * kTcPRow;  // packed bytes per stage: 8 KB
 constexpr int kTcBox = 32;              // output box: 32 tokens x 32 weight rows
 constexpr int kTcEpiBufs = 2;          // 4 KB output staging buffers per epilogue warp
 
@@ -85,20 +82,25 @@ struct GemmTcArgs {
 // output boxes (4 warps x kTcEpiBufs x 4 KB), mbarriers, the tensor-memory base and the
 // abort flag.  Tensor memory: two accumulators of BT columns, then SC code
 // stages of 64 columns (256 k).
-template <int BT, int SA, int SC, int SP>
+template <int BT, int SA, int SC, int SP, int SK>
 struct TcSmem {
+    static_assert(SK == 256 || SK == 512, "k per stage");
+    static constexpr int kABoxes = SK / kTcBK;                   // activation boxes per stage
+    static constexpr int kPRow = SK / 4;                         // packed bytes of a weight row per stage
+    static constexpr int kPChunks = kPRow / 16;                  // its 16-byte chunks (4 or 8)
+    static constexpr int kPStage = kTcRows * kPRow;              // packed bytes per stage
     static constexpr int kAHalf = BT * kTcBK;                    // one activation box
-    static constexpr int kAStage = 2 * kAHalf;
+    static constexpr int kAStage = kABoxes * kAHalf;
     static constexpr int kA = 0;
     static constexpr int kP = kA + SA * kAStage;                 // 1024-aligned (multiples of 1 KB)
-    static constexpr int kE = kP + SP * kTcPStage;
+    static constexpr int kE = kP + SP * kPStage;
     static constexpr int kBars = kE + 4 * kTcEpiBufs * 4096;
     // a_full, a_empty, p_full, p_empty, c_full, c_empty, accum_full x 2, accum_empty x 2, drain
     static constexpr int kBarCount = 2 * SA + 2 * SP + 2 * SC + 5;
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kCodeCol = 2 * BT;                      // first code-stage column
-    static constexpr int kCodeCols = kTcSK / 4;                  // 32-bit columns of one code stage
+    static constexpr int kCodeCols = SK / 4;                     // 32-bit columns of one code stage
     static constexpr int kTmemNeed = 2 * BT + kCodeCols * SC;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
@@ -228,11 +230,11 @@ __device__ __forceinline__ TcUnit tc_unit(const GemmTcArgs &a, int u) {
     return t;
 }
 
-template <int BT, bool BF16_OUT, int SA, int SC, int SP>
+template <int BT, bool BF16_OUT, int SA, int SC, int SP, int SK>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
                         const __grid_constant__ CUtensorMap ymap, const GemmTcArgs a) {
-    using L = TcSmem<BT, SA, SC, SP>;
+    using L = TcSmem<BT, SA, SC, SP, SK>;
     static_assert(BT % 16 == 0 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -299,8 +301,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int ua = blockIdx.x, ka = 0, up = blockIdx.x, kp = 0, ia = 0, ip = 0;
             TcUnit ta = tc_unit(a, ua), tp = ta;
             auto issue_p = [&]() {
-                mbar_arrive_expect_tx(&p_full[ip % SP], kTcPStage);
-                tma_load_2d(sm + L::kP + (ip % SP) * kTcPStage, &pmap, (tp.z * a.sps + kp) * kTcPRow, tp.nt * kTcRows,
+                mbar_arrive_expect_tx(&p_full[ip % SP], L::kPStage);
+                tma_load_2d(sm + L::kP + (ip % SP) * L::kPStage, &pmap, (tp.z * a.sps + kp) * L::kPRow, tp.nt * kTcRows,
                             &p_full[ip % SP]);
                 ++ip;
                 if (++kp == unit_stages(tp)) {
@@ -319,10 +321,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bool issued = false;
                 if (ua < units && (ia < SA || mbar_test_wait(&a_empty[ia % SA], (uint32_t)((ia / SA) - 1) & 1u))) {
                     mbar_arrive_expect_tx(&a_full[ia % SA], L::kAStage);
-                    const int kx = (ta.z * a.sps + ka) * kTcSK;
+                    const int kx = (ta.z * a.sps + ka) * SK;
                     uint8_t *ad = sm + L::kA + (ia % SA) * L::kAStage;
-                    tma_load_2d(ad, &amap, kx, ta.mt * BT, &a_full[ia % SA]);
-                    tma_load_2d(ad + L::kAHalf, &amap, kx + kTcBK, ta.mt * BT, &a_full[ia % SA]);
+#pragma unroll
+                    for (int h = 0; h < L::kABoxes; ++h)
+                        tma_load_2d(ad + h * L::kAHalf, &amap, kx + h * kTcBK, ta.mt * BT, &a_full[ia % SA]);
                     ++ia;
                     if (++ka == unit_stages(ta)) {
                         ka = 0;
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t bs = smem_u32(sm + L::kA + sa * L::kAStage);
                     const uint32_t ac = tmem + (uint32_t)(L::kCodeCol + L::kCodeCols * sc);
 #pragma unroll
-                    for (int kk = 0; kk < kTcSK / 32; ++kk)
+                    for (int kk = 0; kk < SK / 32; ++kk)
                         umma_i8_ts(dt, ac + 8 * kk,
                                    umma_desc_sw128(bs + (kk >> 2) * L::kAHalf + (kk & 3) * 32), idesc,
                                    (kb > 0 || kk > 0) ? 1u : 0u);
@@ -405,7 +408,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int group = (warp - 2) >> 2;       // stages g with g % kTcDecGroups == group
         const int row = quarter * 32 + lane;     // this thread's weight row in a tile
         const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
-        const int sw = (row >> 1) & 3;
+        // packed rows arrive swizzled: 16-byte chunk c of row r at
+        // r * kPRow + ((c ^ ((r >> (3 - log2 kPChunks)) & (kPChunks - 1))) * 16)
+        // (the 64-byte swizzle for 4 chunks, the 128-byte one for 8)
+        const int sw = (row >> (L::kPChunks == 8 ? 0 : 1)) & (L::kPChunks - 1);
         int g = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
@@ -420,31 +426,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                // the packed tile arrives with the 64-byte swizzle: 16-byte chunk c
-                // of row r sits at r * 64 + ((c ^ ((r >> 1) & 3)) * 16)
-                const uint8_t *pr = sm + L::kP + ps * kTcPStage + row * kTcPRow;
-                uint32_t w[16];
+                const uint8_t *pr = sm + L::kP + ps * L::kPStage + row * L::kPRow;
+                uint32_t w[4 * L::kPChunks];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int ch = 0; ch < L::kPChunks; ++ch) {
                     const uint4 p = *reinterpret_cast<const uint4 *>(pr + ((ch ^ sw) << 4));
                     w[4 * ch] = p.x;
                     w[4 * ch + 1] = p.y;
                     w[4 * ch + 2] = p.z;
                     w[4 * ch + 3] = p.w;
                 }
-                uint32_t c[64];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        c[4 * i + j] = (((w[i] >> (2 * j)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
-                }
                 __syncwarp();  // every lane has its packed row in registers
                 if (lane == 0)
                     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&p_empty[ps])) : "memory");
                 const uint32_t cs = tq + (uint32_t)(L::kCodeCol + L::kCodeCols * s);
-                tmem_st32(cs, c);
-                tmem_st32(cs + 32, c + 32);
+                // 16 packed words (256 k) -> 64 code words -> 64 columns at a time
+#pragma unroll
+                for (int gq = 0; gq < L::kPChunks / 4; ++gq) {
+                    uint32_t c[64];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            c[4 * i + j] = (((w[16 * gq + i] >> (2 * j)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
+                    }
+                    tmem_st32(cs + 64 * gq, c);
+                    tmem_st32(cs + 64 * gq + 32, c + 32);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
