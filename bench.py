@@ -324,9 +324,47 @@ def measure_bitlinear_decode(torch, bn, shapes, warmup, l2_bytes, reps=30):
     return out
 
 
+def measure_small_batch(torch, bn, shapes, ms_list, warmup, l2_bytes, reps=30):
+    """Small-batch decode (M tokens, one pass over the weights): int32 GEMM and
+    BitLinear, mean per-call time in a graph of back-to-back calls over
+    rotating weight copies (each copy last read more than 2x L2 earlier)."""
+    out = []
+    for (N, K) in shapes:
+        q1, w = synth.uniform_int8_ternary(N, K, seed=0, M=max(ms_list))
+        packed = bn.bitnet_pack_weights(to_dev(torch, w))
+        del w
+        C = rotation_copies(packed.numel(), l2_bytes)
+        copies = [packed] + [packed.clone() for _ in range(C - 1)]
+        gamma = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+        L = 4 * C
+        for M in ms_list:
+            q = to_dev(torch, q1[:M].copy())
+            x = bf16_dev(torch, synth.bf16_activations(M, K, seed=M, outlier_p=0.01))
+            y = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            ws = bn.workspace(M, N, K)
+            row = {"M": M, "N": N, "K": K}
+            for name, fn in (("int32", lambda i: bn.bitnet_w2a8_gemm(q, copies[i % C], N, y=y, ws=ws)),
+                             ("bitlinear", lambda i: bn.bitnet_bitlinear(x, copies[i % C], gamma, N, y=yb, ws=ws))):
+                def run(fn=fn):
+                    for i in range(L):
+                        fn(i)
+                g = capture(torch, run)
+                ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+                us = ms * 1e3 / (reps * L)
+                nbytes = gemv_bytes(M, N, K) if name == "int32" else bitlinear_bytes(M, N, K)
+                row[f"{name}_us_per_call"] = round(us, 3)
+                row[f"{name}_GBps"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+                del g
+            out.append(row)
+        del copies
+    return out
+
+
 def measure_prefill(torch, bn, ms_list, shapes, warmup, int8_peak_tops, reps=20, L=10):
-    """Prefill GEMM (tcgen05, int32 out): mean per-call time in a graph of L
-    back-to-back calls; int8 TOPS = 2*M*N*K / time."""
+    """Prefill GEMM (tcgen05): mean per-call time in a graph of L back-to-back
+    calls, int32 out (int8 TOPS = 2*M*N*K / time) and the whole BitLinear (bf16
+    in: quantisation pass + GEMM with the bf16 epilogue)."""
     out = []
     for (N, K) in shapes:
         W = synth.bf16_weights(N, K, seed=1)
@@ -348,10 +386,22 @@ def measure_prefill(torch, bn, ms_list, shapes, warmup, int8_peak_tops, reps=20,
             ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
             us = ms * 1e3 / (reps * L)
             tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            del g
+            yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            wsb = bn.workspace(M, N, K)
+
+            def run_bl():
+                for _ in range(L):
+                    bn.bitnet_bitlinear(xd, packed, gamma, N, y=yb, ws=wsb)
+            g = capture(torch, run_bl)
+            ms_bl = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+            us_bl = ms_bl * 1e3 / (reps * L)
+            del g
             out.append({"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "int8_TOPS": round(tops, 1),
                         "frac_int8_peak": round(tops / int8_peak_tops, 4),
-                        "GBps": round(gemv_bytes(M, N, K) / (us * 1e-6) / 1e9, 1)})
-            del g
+                        "GBps": round(gemv_bytes(M, N, K) / (us * 1e-6) / 1e9, 1),
+                        "bitlinear_us_per_call": round(us_bl, 2),
+                        "bitlinear_TOPS": round(2.0 * M * N * K / (us_bl * 1e-6) / 1e12, 1)})
     return out
 
 
@@ -427,6 +477,8 @@ def run_ours(args, rank, world, dist):
         torch.cuda.empty_cache()
         details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
                                                                args.warmup, l2)
+        details["small_batch"] = measure_small_batch(torch, bn, synth.BITLINEAR_DECODE_SHAPES, [2, 4, 8],
+                                                     args.warmup, l2)
         details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES, args.warmup, int8_peak)
         bf = measure_bf16_context(torch, synth.SWEEP_SHAPES, args.warmup, l2)
         for row, ours in zip(bf, details["sweep"]):
