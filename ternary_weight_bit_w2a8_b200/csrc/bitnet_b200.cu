@@ -211,24 +211,34 @@ constexpr int kTmaNumCfg = 5;
 constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
-// Kernel of (mode, warps, tokens per launch).  int8 activations: one token on
-// 4, 8, 12 or 16 warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps.  bf16
-// activations quantised in the kernel: one token only (a batch is quantised
-// once beforehand and takes the int8 kernels).  Slot in the shared-memory
-// opt-in table: MT == 1 ? xmode * 10 + W / 4 - 1 : 4 + 2 * log2(MT / 2) + (W == 16); -1 if none.
+// BitLinear with up to this many tokens quantises them inside the GEMV's
+// prologue (every CTA reads and quantises all of them); more tokens are
+// quantised once by quant_act_kernel first.  Measured on B200, 2560 x 6912:
+// 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
+constexpr int kFusedQuantMaxTokens = 4;
+
+// Kernel of (mode, warps, tokens per launch): one token on 4, 8, 12 or 16
+// warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8 activations
+// (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16 activations
+// quantised in the kernel (xmode 1).  Slot in the shared-memory opt-in table:
+// MT == 1 ? xmode * 10 + W / 4 - 1 : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16);
+// -1 if none.
 int tma_kernel_slot(int xmode, int cfg, int mt) {
     const int W = kTmaCfg[cfg][0];
     if (mt == 1) return xmode * 10 + W / 4 - 1;
-    if (xmode != 0 || (W != 8 && W != 16)) return -1;
-    return 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
+    if (W != 8 && W != 16) return -1;
+    if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
+    return xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
 }
 
 TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
-    static const TmaKernel table[14] = {
+    static const TmaKernel table[20] = {
         gemv_tma_kernel<0, 4, 1>, gemv_tma_kernel<0, 8, 1>, gemv_tma_kernel<0, 12, 1>, gemv_tma_kernel<0, 16, 1>,
         gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 16, 4>,
         gemv_tma_kernel<0, 8, 8>, gemv_tma_kernel<0, 16, 8>,
-        gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>};
+        gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>,
+        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 16, 2>, gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 16, 4>,
+        nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
     const int slot = tma_kernel_slot(xmode, cfg, mt);
     return slot < 0 ? nullptr : table[slot];
 }
@@ -665,8 +675,9 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
         if (tp.use) {
             p.path = kPathGemv;
             p.ws_bytes = tp.ws_bytes;
-            // BitLinear on several tokens quantises them once into the workspace
-            if (bitlinear && M >= 2) p.ws_bytes = round_up(M * K, 256) + round_up(M * 4, 256);
+            // BitLinear on more tokens than the fused prologue takes quantises
+            // them once into the workspace
+            if (bitlinear && M > kFusedQuantMaxTokens) p.ws_bytes = round_up(M * K, 256) + round_up(M * 4, 256);
             return p;
         }
     }
@@ -854,7 +865,7 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    if (p.path == kPathGemv && M >= 2 && M <= 8 && tma_plan(M, N, K).use) {
+    if (p.path == kPathGemv && M > kFusedQuantMaxTokens && M <= 8 && tma_plan(M, N, K).use) {
         // small batch: quantise the tokens once, then one pass over the weights
         int8_t *q = static_cast<int8_t *>(workspace);
         float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * K, 256));
@@ -862,7 +873,7 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         if ((rc = launched()) != BITNET_OK) return rc;
         return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, nullptr, y, s, gamma, nullptr, st);
     }
-    if (p.path == kPathGemv)  // activations quantised per token inside the GEMV: one launch
+    if (p.path == kPathGemv)  // the tokens are quantised inside the GEMV's prologue: one launch
         return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
     // quantise into K_pad-strided rows (zero-padded), then the tensor-core GEMM with the bf16 epilogue
     const int64_t ldq = k_pad(K);

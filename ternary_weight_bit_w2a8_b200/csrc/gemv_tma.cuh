@@ -190,6 +190,62 @@ __device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, floa
     return sc;
 }
 
+// Linear staging with fused quantisation of MT tokens at once (same
+// arithmetic as quant_act_kernel): one pass over every token's row for the
+// absmax values, one block reduction for all of them, then every token is
+// quantised, with slice sums as above.  Token slots t >= M are staged as
+// zeros.  `red` holds MT x 32 floats.
+template <int MT>
+__device__ __forceinline__ void stage_qlin_bf16_tokens(int8_t *qlin, int *qslice, int slices, float *red,
+                                                       const uint16_t *x, int M, int64_t K, int64_t kq,
+                                                       float (&sc)[MT]) {
+    const int64_t npieces = ceil_div(K, 16);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    float am[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) am[t] = 0.0f;
+    for (int64_t p = threadIdx.x; p < npieces; p += blockDim.x) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            if (t < M) {
+                const uint16_t *xr = x + (int64_t)t * K;
+                uint4 lo, hi;
+                load_x16(xr, K, p, (reinterpret_cast<uintptr_t>(xr) & 15) == 0, lo, hi);
+                am[t] = amax16(lo, hi, am[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        float v = am[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[t * 32 + warp] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        float v = 0.0f;
+        for (int w = 0; w < nwarps; ++w) v = fmaxf(v, red[t * 32 + w]);
+        sc[t] = t < M ? __fdiv_rn(127.0f, v > kQuantEps ? v : kQuantEps) : 0.0f;
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        const uint16_t *xr = x + (int64_t)t * K;
+        const bool vec = (reinterpret_cast<uintptr_t>(xr) & 15) == 0;
+        for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < M && p < npieces) {
+                uint4 lo, hi;
+                load_x16(xr, K, p, vec, lo, hi);
+                quant16(lo, hi, sc[t], v);
+            }
+            *reinterpret_cast<uint4 *>(qlin + t * kq + p * 16) = v;
+            slice_sum(qslice + t * slices, p, v);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ kernel
 
 // Resident CTAs the register budget leaves room for: two for the 8-warp and
@@ -202,9 +258,9 @@ template <int XMODE, int W, int MT>
 __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
     static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8, "tokens per launch");
-    static_assert(XMODE == 0 || MT == 1, "bf16 activations: one token per launch");
+
     extern __shared__ uint8_t smem_raw[];
-    __shared__ float red[32];
+    __shared__ float red[(XMODE == 1 ? MT : 1) * 32];
     // the descriptor fetch is the first long latency of the launch: start it now
     if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     const int ns = a.ns, slices = a.slices;
@@ -268,8 +324,10 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     pdl_wait();
 
     float sc[MT];
+    if (XMODE == 1 && MT > 1) stage_qlin_bf16_tokens<MT>(qlin, qslice, slices, red, a.x, a.M, a.K, kq, sc);
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
+        if (XMODE == 1 && MT > 1) break;  // staged above
         sc[t] = 0.0f;
         int8_t *qt = qlin + t * kq;
         int *qst = qslice + t * slices;
