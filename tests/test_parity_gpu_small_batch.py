@@ -32,7 +32,10 @@ def test_small_batch_int32_exact(M, N, K):
     assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w))
 
 
-@pytest.mark.parametrize("M,N,K", [(2, 500, 2560), (3, 6912, 2560), (8, 2560, 6912)])
+# 2..4 tokens are quantised inside the GEMV prologue, 5..8 in a pass of their
+# own first: both sides of that boundary are here
+@pytest.mark.parametrize("M,N,K", [(2, 500, 2560), (3, 6912, 2560), (4, 257, 1536), (5, 300, 3200),
+                                   (8, 2560, 6912)])
 def test_small_batch_bitlinear(M, N, K):
     x, W = synth.bitlinear_inputs(M, N, K, seed=M)
     x[1] = 0  # a zero token among them
