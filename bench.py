@@ -161,8 +161,14 @@ def replay_steps(graphs, n, multi=None):
 
 
 def timed_graph_loop(torch, graphs, steps, warmup, dist=None, multi=None):
-    """`warmup` untimed steps, then exactly `steps` timed ones (see replay_steps).
-    Returns the elapsed ms (max over ranks)."""
+    """Every graph replayed once (so the first replay's one-time cost never
+    lands in the timed region, whatever `warmup` is), `warmup` untimed steps,
+    then exactly `steps` timed ones (see replay_steps).  Returns the elapsed ms
+    (max over ranks)."""
+    if multi is not None:
+        multi.replay()
+    for g in graphs:
+        g.replay()
     replay_steps(graphs, warmup, multi)
     torch.cuda.synchronize()
     if dist is not None:
@@ -292,6 +298,51 @@ def e2e_sweep(torch, bn, gs, steps):
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     return ms, h2d, d2h
+
+
+E2E_SRC = os.path.join(ROOT, "bench_e2e.cu")
+E2E_LIB = os.path.join(ROOT, "bench_e2e.so")
+
+
+def build_e2e():
+    """Compiles bench_e2e.cu (the C loop of the end-to-end leg) if needed."""
+    if not os.path.exists(E2E_LIB) or os.path.getmtime(E2E_LIB) < os.path.getmtime(E2E_SRC):
+        subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17", "-shared",
+                        "-Xcompiler", "-fPIC", "--cudart", "static",
+                        "-o", E2E_LIB + ".tmp", E2E_SRC, "-ldl"], check=True)
+        os.replace(E2E_LIB + ".tmp", E2E_LIB)
+    return E2E_LIB
+
+
+def e2e_sweep_c(torch, bn, gs, steps):
+    """The end-to-end sweep of e2e_sweep driven from C (bench_e2e.cu): the same
+    copies and bitnet_w2a8_gemm calls with no interpreter between them."""
+    import ctypes
+    lib = ctypes.CDLL(build_e2e())
+    fn = lib.e2e_sweep_loop
+    fn.restype = ctypes.c_double
+    P = ctypes.c_void_p
+    fn.argtypes = [ctypes.c_char_p, ctypes.c_int, P, P, P, P, P, ctypes.c_int, P, P, P, P, ctypes.c_int, P,
+                   ctypes.POINTER(ctypes.c_int)]
+    S = len(gs.shapes)
+    hq = [q.cpu().pin_memory() for q in gs.q]
+    hy = [torch.empty(y.shape, dtype=torch.int32).pin_memory() for y in gs.y]
+    arr = lambda ts: (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])  # noqa: E731
+    Ns = (ctypes.c_int64 * S)(*[N for N, _ in gs.shapes])
+    Ks = (ctypes.c_int64 * S)(*[K for _, K in gs.shapes])
+    packed = arr([p for cp in gs.copies for p in cp])
+    wsb = (ctypes.c_int64 * S)(*[w.numel() for w in gs.ws])
+    status = ctypes.c_int(0)
+    args = [bn.LIB_PATH.encode(), S, Ns, Ks, arr(hq), arr(gs.q), packed, len(gs.copies), arr(gs.y), arr(hy),
+            arr(gs.ws), wsb]
+    stream = torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    if fn(*args, 3, stream, ctypes.byref(status)) < 0:
+        raise RuntimeError(f"e2e C loop failed (library status {status.value})")
+    ms = fn(*args, steps, stream, ctypes.byref(status))
+    if ms < 0:
+        raise RuntimeError(f"e2e C loop failed (library status {status.value})")
+    return ms
 
 
 def measure_bitlinear_decode(torch, bn, shapes, warmup, l2_bytes, reps=30):
@@ -459,6 +510,8 @@ def run_ours(args, rank, world, dist):
     e2e_ms, h2d, d2h = e2e_sweep(torch, bn, gs, e2e_steps)
     e2e_ms = max_over_ranks(torch, e2e_ms, dist, "cuda")
     e2e_value = job_gbps(gs.bytes_per_step, e2e_steps, e2e_ms, world)
+    e2e_c_ms = max_over_ranks(torch, e2e_sweep_c(torch, bn, gs, e2e_steps), dist, "cuda")
+    e2e_c_value = job_gbps(gs.bytes_per_step, e2e_steps, e2e_c_ms, world)
 
     details = {"sweep": [{"N": N, "K": K, "us_per_call": round(u, 3),
                           "GBps": round(gemv_bytes(1, N, K) / (u * 1e-6) / 1e9, 1),
@@ -477,7 +530,7 @@ def run_ours(args, rank, world, dist):
         torch.cuda.empty_cache()
         details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
                                                                args.warmup, l2)
-        details["small_batch"] = measure_small_batch(torch, bn, synth.BITLINEAR_DECODE_SHAPES, [2, 4, 8],
+        details["small_batch"] = measure_small_batch(torch, bn, synth.BITLINEAR_DECODE_SHAPES, [2, 4, 8, 16, 32, 64],
                                                      args.warmup, l2)
         details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES, args.warmup, int8_peak)
         bf = measure_bf16_context(torch, synth.SWEEP_SHAPES, args.warmup, l2)
@@ -507,7 +560,7 @@ def run_ours(args, rank, world, dist):
                    "seed": "rank"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                     "traffic_source": "profiles/traffic_gemv_tma_sweep.md (ncu dram__bytes_read.sum + "
+                     "traffic_source": "profiles/traffic_gemv_tma_sweep.json (ncu dram__bytes_read.sum + "
                                        "dram__bytes_write.sum, mean over the 8 sweep launches); null when the "
                                        "kernel sources changed since that capture",
                      "kernel": "gemv_tma_kernel", "peak_source": peaks["source"],
@@ -518,7 +571,12 @@ def run_ours(args, rank, world, dist):
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
                 "note": "public API calls with pinned host activations copied in and int32 results copied out "
-                        "every step, stream synchronised per step; packed weights resident"},
+                        "every step, stream synchronised per step; packed weights resident",
+                "c_loop": {"value": round(e2e_c_value, 2), "unit": "GB/s",
+                           "us_per_step": round(e2e_c_ms * 1e3 / e2e_steps, 2),
+                           "note": "the same copies and C-ABI calls driven from C (bench_e2e.cu): library and "
+                                   "runtime overhead without the Python binding"},
+                "python_us_per_step": round(e2e_ms * 1e3 / e2e_steps, 2)},
         "gpu_launches": int(launches_per_step * args.steps),
         "device_error": err,
         "details": details,
@@ -544,6 +602,19 @@ def oracle_sweep_step(shapes_data, frac, step):
 def cpu_threads():
     n = os.environ.get("OMP_NUM_THREADS")
     return int(n) if n else (os.cpu_count() or 1)
+
+
+def cpu_baseline_one_thread(budget_s=4.0):
+    """The same oracle sample on one host thread: a child process with
+    OMP_NUM_THREADS=1 (the OpenMP thread count is fixed when a process first
+    uses it)."""
+    env = dict(os.environ)
+    env["OMP_NUM_THREADS"] = "1"
+    r = subprocess.run([sys.executable, os.path.abspath(__file__), "--cpu-baseline-only",
+                        "--cpu-budget", str(budget_s)], env=env, capture_output=True, text=True, timeout=600)
+    if r.returncode != 0:
+        return {"error": r.stderr.strip().splitlines()[-1:] or ["failed"]}
+    return json.loads(r.stdout.strip().splitlines()[-1])
 
 
 def cpu_baseline(budget_s=4.0):
@@ -601,7 +672,7 @@ def run_reference(args):
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "traffic_gemv_tma_sweep.md")
+TRAFFIC_DATA = os.path.join(ROOT, "profiles", "traffic_gemv_tma_sweep.json")
 TRAFFIC_SOURCES = ("common.cuh", "quant.cuh", "gemv.cuh", "gemv_tma.cuh")
 # the tensor-core GEMM's section of the translation unit (not part of the GEMV)
 TC_SECTION = ("// ------------------------------------------------------------------ tcgen05 GEMM (M > 1)",
@@ -627,25 +698,24 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
-def read_traffic(path=TRAFFIC_SUMMARY):
+def read_traffic(path=TRAFFIC_DATA):
     """DRAM bytes per launch (read + write, mean over the sweep's launches) from
-    the committed ncu summary, or None when the kernel sources changed since."""
+    the committed ncu capture's data file, or None when the kernel sources
+    changed since that capture."""
     if not os.path.exists(path):
         return None
-    fields = {}
     with open(path) as f:
-        for line in f:
-            key = line.split(":", 1)[0].strip()
-            if ":" in line and key in ("source_sha256", "traffic_bytes_per_launch"):
-                fields[key] = line.split(":", 1)[1].strip().strip("`")
-    if fields.get("source_sha256") != kernel_source_hash() or "traffic_bytes_per_launch" not in fields:
+        d = json.load(f)
+    if d.get("source_sha256") != kernel_source_hash() or d.get("traffic_bytes_per_launch") is None:
         return None
-    return float(fields["traffic_bytes_per_launch"])
+    return float(d["traffic_bytes_per_launch"])
 
 
 def run_profile(args):
-    """`warmup + steps` plain calls over rotating weight copies, no graphs: of one
-    problem (M,N,K), or with `sweep` of each sweep shape at M = 1, in order."""
+    """`warmup + steps` plain calls, no graphs: the int32 contraction of one
+    problem (M,N,K) over rotating weight copies, of each sweep shape at M = 1
+    in order (`sweep`), the activation quantisation (`quant,M,K`) or the
+    BitLinear forward (`bitlinear,M,N,K`)."""
     import torch
     import ternary_weight_bit_w2a8_b200 as bn
     if args.profile == "sweep":
@@ -657,7 +727,31 @@ def run_profile(args):
         print(json.dumps({"profile": "sweep", "calls": (args.warmup + args.steps) * len(gs.shapes),
                           "device_error": bn.bitnet_get_device_error()}))
         return 0
-    M, N, K = (int(v) for v in args.profile.split(","))
+    parts = args.profile.split(",")
+    if parts[0] in ("quant", "bitlinear"):
+        # bf16 activations: the quantisation pass alone (quant,M,K) or the whole
+        # BitLinear forward (bitlinear,M,N,K), weights ternarised on the GPU
+        M, K = int(parts[1]), int(parts[-1])
+        x = bf16_dev(torch, synth.bf16_activations(M, K, seed=0, outlier_p=0.0))
+        if parts[0] == "quant":
+            q, s, r = bn.bitnet_quant_act(x)
+            fn = lambda: bn.bitnet_quant_act(x, q=q, s=s, rowsum=r)  # noqa: E731
+        else:
+            N = int(parts[2])
+            Wd = bf16_dev(torch, synth.bf16_weights(N, K, seed=1))
+            gamma = bn.bitnet_absmean(Wd)
+            packed = bn.bitnet_pack_weights(bn.bitnet_ternarize(Wd, gamma))
+            del Wd
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            ws = bn.workspace(M, N, K)
+            fn = lambda: bn.bitnet_bitlinear(x, packed, gamma, N, y=y, ws=ws)  # noqa: E731
+        for _ in range(args.warmup + args.steps):
+            fn()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": parts, "calls": args.warmup + args.steps,
+                          "device_error": bn.bitnet_get_device_error()}))
+        return 0
+    M, N, K = (int(v) for v in parts)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     gen = synth.sparse_ternary_normal_int8 if (N, K) in synth.LARGE_SHAPES else synth.uniform_int8_ternary
     q, w = gen(N, K, seed=0, M=M)
@@ -686,9 +780,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work for the whole --impl reference run")
-    ap.add_argument("--profile", metavar="M,N,K|sweep",
-                    help="profiling mode: only plain bitnet_w2a8_gemm calls, `warmup + steps` of one problem "
-                         "or of each sweep shape (for ncu)")
+    ap.add_argument("--cpu-baseline-only", action="store_true",
+                    help="print the oracle's CPU baseline (the threads OMP_NUM_THREADS allows) and exit")
+    ap.add_argument("--cpu-budget", type=float, default=4.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--profile", metavar="M,N,K|sweep|quant,M,K|bitlinear,M,N,K",
+                    help="profiling mode (for ncu): `warmup + steps` plain calls of bitnet_w2a8_gemm on one "
+                         "problem or on each sweep shape, of bitnet_quant_act, or of bitnet_bitlinear")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -696,6 +793,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.cpu_baseline_only:
+        print(json.dumps(cpu_baseline(args.cpu_budget)), flush=True)
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
@@ -720,7 +821,9 @@ def main():
     try:
         res = run_ours(args, rank, world, dist)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline()
+            res["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+            res["cpu_baseline"]["host_cpu_count"] = os.cpu_count()
+            res["cpu_baseline"]["one_thread"] = cpu_baseline_one_thread(args.cpu_budget)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

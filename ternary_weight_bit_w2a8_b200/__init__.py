@@ -77,14 +77,14 @@ def _check(rc: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream=None):
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream
 
 
 def _dev(t, name):

@@ -37,8 +37,8 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[22] = {};  // dynamic shared memory opted into by each TMA GEMV variant
-    bool tc_attr_set[10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
+    size_t tma_max_dyn[32] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    bool tc_attr_set[2 * 10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
     OccEntry occ[kOccCache];     // resident CTAs per SM by (instantiation, shared memory)
@@ -105,6 +105,36 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// ------------------------------------------------------------------ per-call tags
+// Kernels whose CTAs meet through counters or flags in the workspace tag
+// them with a per-call value, so that no zeroing is needed (see gemv_tma.cuh
+// and gemm_tc.cuh).  The top nibble 0xA keeps every tag outside the range of
+// the int32 partial sums (|sum| < 2^28) that share the workspace.
+std::atomic<uint32_t> g_epoch{1};
+inline uint32_t next_epoch() { return 0xA0000000u | (g_epoch.fetch_add(1, std::memory_order_relaxed) & 0x0FFFFFFFu); }
+
+// ------------------------------------------------------------------ activation quantisation
+// Teams of 1..8 warps per token: about a thousand warps in flight whatever M
+// (one warp per token from 1024 tokens up), so the pass is one wave that reads
+// each row from HBM once.
+int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_t *q, int64_t ldq, bool zero_pad,
+                 float *s, int32_t *rowsum, cudaStream_t st) {
+    const int wpt = M >= 1024 ? 1 : (M >= 512 ? 2 : (M >= 256 ? 4 : 8));
+    const int64_t teams_per_cta = kThreads / (32 * wpt);
+    int64_t grid = ceil_div(M, teams_per_cta);
+    const int64_t cap = (int64_t)dev->sm_count * (2048 / kThreads);
+    if (grid > cap) grid = cap;
+    const dim3 g((unsigned)grid), b(kThreads);
+    cudaError_t e;
+    switch (wpt) {
+        case 1: e = launch_pdl(quant_act_kernel<1>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        case 2: e = launch_pdl(quant_act_kernel<2>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        case 4: e = launch_pdl(quant_act_kernel<4>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        default: e = launch_pdl(quant_act_kernel<8>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+    }
+    return launched(e);
+}
+
 // ------------------------------------------------------------------ fill (K == 0)
 template <typename T>
 __global__ void __launch_bounds__(kThreads) fill_kernel(T *p, int64_t n, T v) {
@@ -119,8 +149,12 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
-struct GemvTune {  // optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns"
-    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0;
+// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,split,warps,fuse"
+// (register GEMV: G, R, U, ctas, prefetch, S; tensor-core GEMM: R < 0 token
+// tile, S K-splits, fuse = 0 quantises BitLinear activations in a pass of
+// their own; TMA GEMV: tma = 0 off, ns ring depth, split -1/0/1, warps)
+struct GemvTune {
+    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, split = -1, warps = 0, fuse = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -129,7 +163,8 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma, &t.ns);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma,
+                   &t.ns, &t.split, &t.warps, &t.fuse);
     });
     return t;
 }
@@ -205,53 +240,105 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 
-// TMA GEMV variants: (warps per CTA, most boxes in flight per warp); the
-// ring depth of a launch is the smaller of the latter and what its items need
-constexpr int kTmaNumCfg = 5;
-constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
+// 2-D tensor maps (inner dimension d0 contiguous, rows of `stride` bytes),
+// encoded once per distinct argument set and kept in a small cache: a map is
+// a pure function of its arguments, so a cached one stays valid for any
+// allocation that reuses the address.  Returns false if encoding fails.
+struct MapKey {
+    const void *ptr;
+    uint64_t d0, d1, stride;
+    uint32_t b0, b1;
+    int dtype, swizzle, promo;
+    bool operator==(const MapKey &o) const {
+        return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 && b1 == o.b1 &&
+               dtype == o.dtype && swizzle == o.swizzle && promo == o.promo;
+    }
+};
+constexpr int kMapCache = 64;
+struct MapCache {
+    MapKey key[kMapCache];
+    CUtensorMap map[kMapCache];
+    int n = 0, next = 0;
+};
+MapCache g_maps[kMaxDevices];
+std::mutex g_maps_mu;
+
+bool encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *ptr, uint64_t d0, uint64_t d1,
+               uint64_t stride, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swizzle,
+               CUtensorMapL2promotion promo) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    const MapKey k{ptr, d0, d1, stride, b0, b1, (int)dtype, (int)swizzle, (int)promo};
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mu);
+        MapCache &c = g_maps[dev];
+        for (int i = 0; i < c.n; ++i)
+            if (c.key[i] == k) {
+                *out = c.map[i];
+                return true;
+            }
+    }
+    if (tensor_map_encoder() == nullptr) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)d0, (cuuint64_t)d1};
+    const cuuint64_t gstride[1] = {(cuuint64_t)stride};
+    const cuuint32_t box[2] = {b0, b1};
+    const cuuint32_t es[2] = {1, 1};
+    if (tensor_map_encoder()(out, dtype, 2, const_cast<void *>(ptr), gdim, gstride, box, es,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lk(g_maps_mu);
+    MapCache &c = g_maps[dev];
+    const int slot = c.n < kMapCache ? c.n++ : c.next;
+    if (slot == c.next) c.next = (c.next + 1) % kMapCache;
+    c.key[slot] = k;
+    c.map[slot] = *out;
+    return true;
+}
+
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
 // BitLinear with up to this many tokens quantises them inside the GEMV's
 // prologue (every CTA reads and quantises all of them); more tokens are
-// quantised once by quant_act_kernel first.  Measured on B200, 2560 x 6912:
+// quantised once by the quantisation pass first.  Measured on B200, 2560 x 6912:
 // 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
 constexpr int kFusedQuantMaxTokens = 4;
 
-// Kernel of (mode, warps, tokens per launch): one token on 4, 8, 12 or 16
-// warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8 activations
-// (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16 activations
-// quantised in the kernel (xmode 1).  Slot in the shared-memory opt-in table:
-// MT == 1 ? xmode * 10 + W / 4 - 1 : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16);
-// -1 if none.
-int tma_kernel_slot(int xmode, int cfg, int mt) {
-    const int W = kTmaCfg[cfg][0];
-    if (mt == 1) return xmode * 10 + W / 4 - 1;
-    if (W != 8 && W != 16) return -1;
-    if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
-    return xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
+// Kernel of (mode, warps, tokens per launch): 4, 8, 12 or 16 warps for one or
+// two tokens, 4 or 8 warps for four or eight (the registers of two CTAs per
+// SM), int8 activations (xmode 0) or, up to kFusedQuantMaxTokens tokens, bf16
+// activations quantised in the kernel (xmode 1).  Index in the kernel and
+// shared-memory opt-in tables, -1 if there is no such kernel.
+int tma_kernel_slot(int xmode, int W, int mt) {
+    const int wi = W == 4 ? 0 : (W == 8 ? 1 : (W == 12 ? 2 : (W == 16 ? 3 : -1)));
+    const int mi = mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : (mt == 8 ? 3 : -1)));
+    if (wi < 0 || mi < 0 || (mt >= 4 && W > 8) || (xmode == 1 && mt > kFusedQuantMaxTokens)) return -1;
+    return xmode * 16 + mi * 4 + wi;
 }
 
-TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
-    static const TmaKernel table[20] = {
+TmaKernel tma_kernel_for(int xmode, int W, int mt) {
+    static const TmaKernel table[32] = {
         gemv_tma_kernel<0, 4, 1>, gemv_tma_kernel<0, 8, 1>, gemv_tma_kernel<0, 12, 1>, gemv_tma_kernel<0, 16, 1>,
-        gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 16, 4>,
-        gemv_tma_kernel<0, 8, 8>, gemv_tma_kernel<0, 16, 8>,
+        gemv_tma_kernel<0, 4, 2>, gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 12, 2>, gemv_tma_kernel<0, 16, 2>,
+        gemv_tma_kernel<0, 4, 4>, gemv_tma_kernel<0, 8, 4>, nullptr, nullptr,
+        gemv_tma_kernel<0, 4, 8>, gemv_tma_kernel<0, 8, 8>, nullptr, nullptr,
         gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>,
-        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 16, 2>, gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 16, 4>,
-        nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
-    const int slot = tma_kernel_slot(xmode, cfg, mt);
+        gemv_tma_kernel<1, 4, 2>, gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 12, 2>, gemv_tma_kernel<1, 16, 2>,
+        gemv_tma_kernel<1, 4, 4>, gemv_tma_kernel<1, 8, 4>, nullptr, nullptr,
+        nullptr, nullptr, nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
+    const int slot = tma_kernel_slot(xmode, W, mt);
     return slot < 0 ? nullptr : table[slot];
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int W, int mt) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    const int si = tma_kernel_slot(xmode, cfg, mt);
+    const int si = tma_kernel_slot(xmode, W, mt);
     if (si < 0) return 0;
     size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, cfg, mt);
+        TmaKernel kern = tma_kernel_for(xmode, W, mt);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -262,72 +349,78 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
 }
 
 // Plan of the TMA GEMV, from the shape and B200 reference figures only (148
-// SMs, 227 KB of shared memory per CTA), so that what a shape needs does not
+// SMs, 228 KB of shared memory per SM), so that what a shape needs does not
 // depend on the device that runs it.
+//   - One CTA per SM (grid = min(items, 148)).  A CTA takes under half an SM
+//     (registers by the kernel's launch bounds, shared memory here), so the
+//     next launch's CTA is resident beside it and requests its weights while
+//     this launch finishes (programmatic dependent launch).
+//   - Whole row blocks per CTA, or, where that leaves the busiest SM more
+//     than kTmaSplitGainItems items above an even share, an even split of
+//     all (row block, K-slice) items: a row block then spans CTAs, whose
+//     int32 partial sums meet in the workspace (see gemv_tma.cuh).
+//   - Warps and ring depth: the most boxes in flight that leave room for a
+//     second CTA; 16 warps when each takes at most one box, else 12 (8 for
+//     four and eight tokens).
+constexpr int kTmaSplitGainItems = 8;
+
 struct TmaPlan {
     bool use;
-    int cfg, slices, max_blocks, grid;
-    int ns;            // ring depth per warp
-    int mt;            // tokens per launch (1, 2, 4, 8)
+    int W, ns, mt, grid, split, slices, max_slots;
+    int64_t nblocks;
     size_t smem;
-    int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
+    int64_t ws_bytes;  // split: partial-sum records and their flags
 };
 
 TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
-    constexpr size_t kRefSmemOptin = 232448;
+    constexpr size_t kRefSmemOptin = 232448;  // one CTA per SM
+    constexpr size_t kRefSmemHalf = 114688;   // two CTAs per SM (1 KB reserved and static memory each)
+    const GemvTune &tn = gemv_tune();
     TmaPlan p{};
-    const int tune = gemv_tune().tma;
-    if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
+    if (M < 1 || M > 8 || tn.tma == 0 || K < kTmaSliceK || N < 1) return p;
+    // a lane accumulates one row's whole K: |acc_j| <= 4096 * K_pad stays
+    // inside int32 for K_pad <= 2^19 (shared memory caps K lower still)
+    if (k_pad(K) > ((int64_t)1 << 19)) return p;
     p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
-    const int64_t row_bytes = packed_row_bytes(K);
-    const int64_t nblocks = ceil_div(N, kTmaRows);
-    p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
-    // variant (measured on B200 over sequences of different shapes, as in a
-    // decode step): 16 x 2, and 12 x 3 for rows of K >= 16384.  Variants that
-    // let two CTAs share an SM win on a shape repeated alone but lose in a
-    // mixed sequence, where the scheduler can then stack two CTAs of one
-    // launch on an SM.
-    if (tune >= 1 && tune <= kTmaNumCfg)
-        p.cfg = tune - 1;
-    else
-        p.cfg = p.slices >= 32 ? 1 : 2;
-    if (p.mt > 1 && kTmaCfg[p.cfg][0] != 8 && kTmaCfg[p.cfg][0] != 16) p.cfg = 2;  // several tokens: 8 or 16 warps
-    const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
-    // at most one CTA per SM per launch (BITNET_GEMV_TUNE's ctas field
-    // overrides): each SM keeps room for a CTA of the next launch, which then
-    // starts and requests its weights while this one finishes
-    const int per_sm = gemv_tune().ctas > 0 ? gemv_tune().ctas : 1;
-    const int64_t gmax = (int64_t)kRefSMs * per_sm;
-    p.grid = (int)(nblocks < gmax ? nblocks : gmax);
-    p.max_blocks = (int)ceil_div(nblocks, p.grid);
-    // ring depth: no more boxes per warp than its items (a small launch then
-    // needs little shared memory and leaves room beside it)
-    const int64_t ipw = ceil_div((int64_t)p.max_blocks * p.slices, W);
-    p.ns = (int)(ipw < NS ? (ipw < 1 ? 1 : ipw) : NS);
-    if (gemv_tune().ns > 0) p.ns = gemv_tune().ns < NS ? gemv_tune().ns : NS;
-    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_blocks, p.mt);
+    p.nblocks = ceil_div(N, kTmaRows);
+    p.slices = (int)ceil_div(packed_row_bytes(K), kTmaSliceBytes);
+    const int64_t items = p.nblocks * p.slices;
+    p.grid = (int)(items < kRefSMs ? items : kRefSMs);
+    const int64_t whole = ceil_div(p.nblocks, p.grid) * p.slices;
+    const int64_t even = ceil_div(items, p.grid);
+    p.split = (whole - even > kTmaSplitGainItems) ? 1 : 0;
+    if (tn.split >= 0) p.split = tn.split;
+    const int64_t ipc = p.split ? even : whole;  // most items of one CTA
+    p.max_slots = (int)(p.split ? (ipc - 1) / p.slices + 2 : ceil_div(p.nblocks, p.grid));
+    int W = p.mt >= 4 ? 8 : (ipc <= 16 ? 16 : 12);
+    if (tn.warps > 0 && tma_kernel_slot(0, tn.warps, p.mt) >= 0) W = tn.warps;
+    // ring depth: as deep as the items need and two CTAs per SM allow
+    const size_t fixed = gemv_tma_smem_bytes(W, 0, p.slices, p.max_slots, p.mt);
+    int64_t ns = ceil_div(ipc, W);
+    if (ns > 4) ns = 4;
+    while (ns > 1 && fixed + (size_t)W * ns * (kTmaBoxBytes + 8) > kRefSmemHalf) --ns;
+    if (tn.ns > 0) ns = tn.ns;
+    p.ns = (int)ns;
+    p.W = W;
+    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_slots, p.mt);
     if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
+    p.ws_bytes = p.split ? round_up((int64_t)p.grid * p.mt * kTmaRows * 4, 256) + round_up((int64_t)p.grid * 4, 256) : 0;
     p.use = true;
     return p;
 }
 
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
-                    const TmaPlan &tp, cudaStream_t st) {
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
+                    const TmaPlan &tp, void *ws, cudaStream_t st) {
+    TmaKernel kern = tma_kernel_for(xmode, tp.W, tp.mt);
     if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
-    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt))
+    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.W, tp.mt))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
-    const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
-    const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kTmaSliceBytes, (cuuint32_t)kTmaRows};
-    const cuuint32_t estride[2] = {1, 1};
-    if (tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
-                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!encode_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes,
+                   kTmaSliceBytes, kTmaRows, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
         return BITNET_ERR_CUDA;
     // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
     // makes one wait run out, exercising the device-timeout path
@@ -346,16 +439,23 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.N = N;
     a.K = K;
     a.slices = tp.slices;
-    a.blk_begin = 0;
-    a.nblocks = ceil_div(N, kTmaRows);
-    a.max_blocks_cta = tp.max_blocks;
+    a.nblocks = tp.nblocks;
+    a.split = tp.split;
+    a.max_slots = tp.max_slots;
     a.ns = tp.ns;
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
     a.s_act = s_act;
+    if (tp.split) {
+        a.rec = static_cast<int32_t *>(ws);
+        a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) +
+                                               round_up((int64_t)tp.grid * tp.mt * kTmaRows * 4, 256));
+        // a tag no int32 partial sum of this library reaches (|sum| < 2^28)
+        a.epoch = next_epoch();
+    }
     a.test_stall = test_stall;
-    return launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
+    return launched(launch_pdl(kern, dim3(tp.grid), dim3(tp.W * 32), tp.smem, st, map, a));
 }
 
 // xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
@@ -366,7 +466,7 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     {
         const TmaPlan tp = tma_plan(M, N, K);
         if (tp.use && ldq == K)
-            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, st);
+            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, ws, st);
     }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();
@@ -460,35 +560,45 @@ int noalloc_scratch(void **out) {
 }
 
 // ------------------------------------------------------------------ tcgen05 GEMM (M > 1)
-// Token-tile widths (UMMA N) of the persistent tensor-core GEMM.
-constexpr int kTcNumBT = 5;
-constexpr int kTcBTs[kTcNumBT] = {192, 128, 64, 32, 16};
+// Token-tile widths (UMMA N) of the persistent tensor-core GEMM.  The first
+// kTcNumPlanned are the planner's candidates (widest first); the rest are
+// reached through the tuning override only.
+constexpr int kTcNumBT = 10;
+constexpr int kTcNumPlanned = 5;
+constexpr int kTcBTs[kTcNumBT] = {192, 128, 64, 32, 16, 128, 96, 64, 128, 192};
 // k per stage of each variant (its packed rows are k / 4 bytes, 64-byte or
 // 128-byte swizzled; its code stages k / 4 tensor-memory columns)
-constexpr int kTcSKs[kTcNumBT] = {256, 512, 256, 256, 256};
+constexpr int kTcSKs[kTcNumBT] = {256, 512, 256, 256, 256, 256, 256, 256, 256, 256};
 // Time of one stage of each variant with every SM busy, measured on B200 (us):
 // the MMA time for the wide tiles, the decoder-to-tensor-core hand-over
 // (~0.6 us) for the narrow ones.
-constexpr double kTcStageUs[kTcNumBT] = {0.69, 1.12, 0.60, 0.60, 0.60};
+constexpr double kTcStageUs[kTcNumBT] = {0.69, 1.12, 0.60, 0.60, 0.60, 0.60, 0.60, 0.60, 0.60, 0.69};
 using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmTcArgs);
 
-// Rings (activation, code, packed stages) per token-tile width.  The 192-,
-// 128- and 64-token variants take all 512 tensor-memory columns (2
-// accumulators + code stages) and more than half an SM's shared memory, so
-// one CTA per SM; the narrower ones take 256 columns.
+// Rings (activation, code, packed stages) per variant.  The 192-, 128- and
+// 64-token variants take all 512 tensor-memory columns (2 accumulators + code
+// stages) and more than half an SM's shared memory, so one CTA per SM; the
+// narrower ones take 256 columns.  The next three trade accumulator width for
+// code stages (4, 5 and 6 in flight instead of 2); the last two keep a single
+// accumulator (no overlap of a unit's epilogue with the next unit) for 6 and
+// 5 code stages.
+#define BITNET_TC_VARIANTS(OUT)                                                                                      \
+    gemm_w2a8_tc_kernel<192, OUT, 3, 2, 4, 256>, gemm_w2a8_tc_kernel<128, OUT, 2, 2, 3, 512>,                      \
+        gemm_w2a8_tc_kernel<64, OUT, 6, 4, 6, 256>, gemm_w2a8_tc_kernel<32, OUT, 8, 3, 6, 256>,                    \
+        gemm_w2a8_tc_kernel<16, OUT, 8, 3, 6, 256>, gemm_w2a8_tc_kernel<128, OUT, 4, 4, 6, 256>,                   \
+        gemm_w2a8_tc_kernel<96, OUT, 5, 5, 6, 256>, gemm_w2a8_tc_kernel<64, OUT, 6, 6, 8, 256>,                    \
+        gemm_w2a8_tc_kernel<128, OUT, 4, 6, 6, 256, 1>, gemm_w2a8_tc_kernel<192, OUT, 3, 5, 4, 256, 1>
 TcKernel tc_kernel_for(int bt_idx, bool bf16, size_t *smem) {
-    static const TcKernel k[2 * kTcNumBT] = {
-        gemm_w2a8_tc_kernel<192, false, 3, 2, 4, 256>, gemm_w2a8_tc_kernel<128, false, 2, 2, 3, 512>,
-        gemm_w2a8_tc_kernel<64, false, 6, 4, 6, 256>,  gemm_w2a8_tc_kernel<32, false, 8, 3, 6, 256>,
-        gemm_w2a8_tc_kernel<16, false, 8, 3, 6, 256>,  gemm_w2a8_tc_kernel<192, true, 3, 2, 4, 256>,
-        gemm_w2a8_tc_kernel<128, true, 2, 2, 3, 512>,  gemm_w2a8_tc_kernel<64, true, 6, 4, 6, 256>,
-        gemm_w2a8_tc_kernel<32, true, 8, 3, 6, 256>,   gemm_w2a8_tc_kernel<16, true, 8, 3, 6, 256>};
+    static const TcKernel k[2 * kTcNumBT] = {BITNET_TC_VARIANTS(false), BITNET_TC_VARIANTS(true)};
     static const size_t raw[kTcNumBT] = {TcSmem<192, 3, 2, 4, 256>::kBytes, TcSmem<128, 2, 2, 3, 512>::kBytes,
-                                         TcSmem<64, 6, 4, 6, 256>::kBytes, TcSmem<32, 8, 3, 6, 256>::kBytes,
-                                         TcSmem<16, 8, 3, 6, 256>::kBytes};
+                                         TcSmem<64, 6, 4, 6, 256>::kBytes,  TcSmem<32, 8, 3, 6, 256>::kBytes,
+                                         TcSmem<16, 8, 3, 6, 256>::kBytes,  TcSmem<128, 4, 4, 6, 256>::kBytes,
+                                         TcSmem<96, 5, 5, 6, 256>::kBytes,  TcSmem<64, 6, 6, 8, 256>::kBytes,
+                                         TcSmem<128, 4, 6, 6, 256, 1>::kBytes, TcSmem<192, 3, 5, 4, 256, 1>::kBytes};
     *smem = raw[bt_idx] + 1024;  // + alignment slack
     return k[(bf16 ? kTcNumBT : 0) + bt_idx];
 }
+#undef BITNET_TC_VARIANTS
 
 // Token-tile width and K-split of the tensor-core GEMM, from a small cost
 // model of the persistent kernel on the B200's 148 SMs (so the workspace a
@@ -511,10 +621,10 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
     TcPlan p{};
     const GemvTune &tn = gemv_tune();
     const int64_t nt = ceil_div(N, kTcRows);
-    int first = kTcNumBT - 1;
+    int first = kTcNumPlanned - 1;
     while (first > 0 && kTcBTs[first] < M) --first;  // smallest tile >= M, else the widest
     double best = 1e30;
-    for (int i = first; i < kTcNumBT; ++i) {
+    for (int i = first; i < kTcNumPlanned; ++i) {
         const int BT = kTcBTs[i];
         const int nk = (int)ceil_div(k_pad(K), kTcSKs[i]);
         const int64_t tiles = nt * ceil_div(M, BT);
@@ -534,7 +644,7 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
             }
         }
     }
-    // tuning overrides: R = -1..-5 picks the token tile, S the split count
+    // tuning overrides: R = -1..-10 picks the variant, S the split count
     if (tn.R < 0 && -tn.R <= kTcNumBT) p.bt_idx = -tn.R - 1;
     const int nk = (int)ceil_div(k_pad(K), kTcSKs[p.bt_idx]);
     if (tn.S > 0) {
@@ -549,9 +659,16 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
 }
 
 // reduce: add int32 results into y_i32 (which the caller has zeroed).
+// BitLinear with the activation quantisation inside the GEMM launch: the bf16
+// activations and the call's counter words (16 bytes of workspace).
+struct TcFuse {
+    const uint16_t *x = nullptr;
+    unsigned long long *sync = nullptr;
+};
+
 int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t *packed, int64_t M, int64_t N,
                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
-                   const TcPlan &tp, int reduce, cudaStream_t st) {
+                   const TcPlan &tp, int reduce, cudaStream_t st, const TcFuse &fuse = TcFuse{}) {
     if (tensor_map_encoder() == nullptr) return BITNET_ERR_CUDA;
     const int bi = tp.bt_idx;
     const int BT = kTcBTs[bi];
@@ -568,26 +685,15 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         }
     }
     CUtensorMap amap, pmap;
-    {
-        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        const cuuint64_t gstride[1] = {(cuuint64_t)lda};
-        const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)BT};
-        const cuuint32_t es[2] = {1, 1};
-        if (tensor_map_encoder()(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(q), gdim, gstride, box,
-                                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return BITNET_ERR_CUDA;
-    }
+    if (!encode_2d(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)K, (uint64_t)M, (uint64_t)lda, kTcBK,
+                   (uint32_t)BT, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+        return BITNET_ERR_CUDA;
     {
         const int64_t row_bytes = packed_row_bytes(K);
-        const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
-        const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-        const cuuint32_t box[2] = {(cuuint32_t)(kTcSKs[bi] / 4), (cuuint32_t)kTcRows};
-        const cuuint32_t es[2] = {1, 1};
-        if (tensor_map_encoder()(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride,
-                                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                 kTcSKs[bi] == 512 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        if (!encode_2d(&pmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)row_bytes, (uint64_t)N,
+                       (uint64_t)row_bytes, (uint32_t)(kTcSKs[bi] / 4), kTcRows,
+                       kTcSKs[bi] == 512 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
             return BITNET_ERR_CUDA;
     }
     // outputs: 32-row boxes of 128 bytes per row, stored through TMA when the
@@ -597,18 +703,12 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     const int esize = bf16 ? 2 : 4;
     void *ybase = bf16 ? static_cast<void *>(y_bf16) : static_cast<void *>(y_i32);
     int tma_store = ((N * esize) % 16 == 0) && aligned(ybase, 16);
-    if (tma_store) {
-        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
-        const cuuint64_t gstride[1] = {(cuuint64_t)(N * esize)};
-        // boxes of 32 weight rows (inner) x up to 32 tokens, unswizzled
-        const cuuint32_t box[2] = {(cuuint32_t)kTcBox, (cuuint32_t)(BT < kTcBox ? BT : kTcBox)};
-        const cuuint32_t es[2] = {1, 1};
-        if (tensor_map_encoder()(&ymap, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_INT32, 2,
-                                 ybase, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            tma_store = 0;
-    }
+    // boxes of 32 weight rows (inner) x up to 32 tokens, unswizzled
+    if (tma_store && !encode_2d(&ymap, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_INT32, ybase,
+                                (uint64_t)N, (uint64_t)M, (uint64_t)(N * esize), kTcBox,
+                                (uint32_t)(BT < kTcBox ? BT : kTcBox), CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE))
+        tma_store = 0;
     GemmTcArgs a{};
     a.M = M;
     a.N = N;
@@ -624,6 +724,13 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
     a.tiles_n = (int)ceil_div(N, kTcRows);
     a.tiles_m = (int)ceil_div(M, BT);
     a.splits = tp.S;
+    if (fuse.x != nullptr) {  // q and s_act are written by this launch
+        a.x = fuse.x;
+        a.qout = const_cast<int8_t *>(q);
+        a.ldq = lda;
+        a.sync = fuse.sync;
+        a.epoch = next_epoch();
+    }
     // persistent: one CTA per SM (or fewer, when there are fewer work units)
     const int64_t units = (int64_t)a.tiles_n * a.tiles_m * a.splits;
     if (units > (int64_t)1 << 30) return BITNET_ERR_UNSUPPORTED;  // work units are counted in int
@@ -676,8 +783,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
             p.path = kPathGemv;
             p.ws_bytes = tp.ws_bytes;
             // BitLinear on more tokens than the fused prologue takes quantises
-            // them once into the workspace
-            if (bitlinear && M > kFusedQuantMaxTokens) p.ws_bytes = round_up(M * K, 256) + round_up(M * 4, 256);
+            // them once into the workspace (before the GEMV's own scratch)
+            if (bitlinear && M > kFusedQuantMaxTokens) p.ws_bytes += round_up(M * K, 256) + round_up(M * 4, 256);
             return p;
         }
     }
@@ -686,8 +793,9 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
         p.tc = tc_plan(M, N, K);
         const int64_t qbytes = round_up(M * k_pad(K), 256);
         if (bitlinear) {
-            // quantised activations, scales and, for a K-split, int32 sums
-            p.ws_bytes = qbytes + round_up(M * 4, 256) + (p.tc.S > 1 ? round_up(M * N * 4, 256) : 0);
+            // quantised activations, scales, the launch's counter words and,
+            // for a K-split, int32 sums
+            p.ws_bytes = qbytes + round_up(M * 4, 256) + 256 + (p.tc.S > 1 ? round_up(M * N * 4, 256) : 0);
         } else {
             p.repack = !q_tma_ok;
             p.ws_bytes = p.repack ? qbytes : 0;
@@ -823,8 +931,7 @@ BITNET_API int bitnet_quant_act(const uint16_t *x, int64_t M, int64_t K, int8_t 
     DeviceInfo *dev = nullptr;
     int rc = device_info(&dev);
     if (rc != BITNET_OK) return rc;
-    quant_act_kernel<<<(unsigned)M, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, K, q, K, false, s, rowsum);
-    return launched();
+    return launch_quant(dev, x, M, K, q, K, false, s, rowsum, static_cast<cudaStream_t>(stream));
 }
 
 BITNET_API int bitnet_w2a8_gemm(const int8_t *q, const uint8_t *packed, int32_t *y, int64_t M, int64_t N, int64_t K,
@@ -869,24 +976,30 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         // small batch: quantise the tokens once, then one pass over the weights
         int8_t *q = static_cast<int8_t *>(workspace);
         float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * K, 256));
-        quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, K, false, s, nullptr);
-        if ((rc = launched()) != BITNET_OK) return rc;
-        return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, nullptr, y, s, gamma, nullptr, st);
+        void *gws = static_cast<char *>(workspace) + round_up(M * K, 256) + round_up(M * 4, 256);
+        if ((rc = launch_quant(dev, x, M, K, q, K, false, s, nullptr, st)) != BITNET_OK) return rc;
+        return launch_gemv(dev, 0, q, nullptr, K, packed, M, N, K, nullptr, y, s, gamma, gws, st);
     }
     if (p.path == kPathGemv)  // the tokens are quantised inside the GEMV's prologue: one launch
         return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
-    // quantise into K_pad-strided rows (zero-padded), then the tensor-core GEMM with the bf16 epilogue
+    // the tensor-core GEMM quantises the rows itself (into K_pad-strided,
+    // zero-padded rows of the workspace) and rescales in its bf16 epilogue
     const int64_t ldq = k_pad(K);
     int8_t *q = static_cast<int8_t *>(workspace);
     float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * ldq, 256));
-    quant_act_kernel<<<(unsigned)M, kThreads, 0, st>>>(x, K, q, ldq, true, s, nullptr);
-    if ((rc = launched()) != BITNET_OK) return rc;
-    if (p.tc.S == 1) return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, p.tc, 0, st);
+    TcFuse fuse;
+    fuse.sync = reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(s) + round_up(M * 4, 256));
+    fuse.x = x;
+    if (gemv_tune().fuse == 0) {  // tuning: a quantisation pass of its own first
+        if ((rc = launch_quant(dev, x, M, K, q, ldq, true, s, nullptr, st)) != BITNET_OK) return rc;
+        fuse.x = nullptr;
+    }
+    if (p.tc.S == 1) return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, p.tc, 0, st, fuse);
     // K-split: int32 sums in the workspace, then the rescale to bf16
-    int32_t *acc = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(s) + round_up(M * 4, 256));
+    int32_t *acc = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(fuse.sync) + 256);
     fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(acc, M * N, 0);
     if ((rc = launched()) != BITNET_OK) return rc;
-    if ((rc = launch_gemm_tc(dev, q, ldq, packed, M, N, K, acc, nullptr, nullptr, nullptr, p.tc, 1, st)) != BITNET_OK)
+    if ((rc = launch_gemm_tc(dev, q, ldq, packed, M, N, K, acc, nullptr, s, nullptr, p.tc, 1, st, fuse)) != BITNET_OK)
         return rc;
     return launched(launch_pdl(rescale_bf16_kernel, dim3(grid_for(M * N, kThreads * 4, dev->sm_count)),
                                dim3(kThreads), (size_t)0, st, (const int32_t *)acc, M, N, (const float *)s, gamma, y));

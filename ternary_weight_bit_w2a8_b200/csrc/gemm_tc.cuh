@@ -76,13 +76,65 @@ struct GemmTcArgs {
     uint16_t *y_bf16;       // [M, N] bf16 result (BitLinear)
     const float *s_act;     // [M] activation scales (BitLinear)
     const float *gamma;     // weight scale (BitLinear)
+    // BitLinear with the quantisation inside this launch (x != null): bf16
+    // activations x [M, K] are quantised by warps 2..13 of every CTA into
+    // qout (rows of ldq bytes, zero-padded: the tensor the activation map
+    // reads) and s_act; sync[0] counts the rows done, sync[1] the CTAs that
+    // finished, both tagged with this call's epoch (see tagged_add)
+    const uint16_t *x;
+    int8_t *qout;
+    int64_t ldq;
+    unsigned long long *sync;
+    uint32_t epoch;
 };
+
+// Adds n to a counter word {tag (high 32 bits) : count (low 32 bits)} and
+// returns the new count.  A word whose tag is not `epoch` (left by an earlier
+// call, or never written) counts from zero, so the counter needs no zeroing;
+// the last user of a call resets it to {epoch, 0} so that a replayed CUDA
+// graph (same epoch) starts from zero too.
+__device__ __forceinline__ uint32_t tagged_add(unsigned long long *w, uint32_t epoch, uint32_t n) {
+    unsigned long long cur = atomicAdd(w, 0ull);
+    for (;;) {
+        const uint32_t tag = (uint32_t)(cur >> 32), c = (uint32_t)cur;
+        const unsigned long long nv = ((unsigned long long)epoch << 32) | (unsigned long long)((tag == epoch ? c : 0u) + n);
+        const unsigned long long prev = atomicCAS(w, cur, nv);
+        if (prev == cur) return (uint32_t)nv;
+        cur = prev;
+    }
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait until the counter holds {epoch, target}; false after the limit
+// or when another role raised the abort flag.
+__device__ __forceinline__ bool wait_tagged(const unsigned long long *w, uint32_t epoch, uint32_t target,
+                                            volatile int *abort_flag) {
+    const unsigned long long want = ((unsigned long long)epoch << 32) | target;
+    if (ld_acquire_u64(w) == want) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (ld_acquire_u64(w) == want) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
 
 // Shared-memory plan: SA activation stages, SP packed stages, the epilogue's
 // output boxes (4 warps x kTcEpiBufs x 4 KB), mbarriers, the tensor-memory base and the
-// abort flag.  Tensor memory: two accumulators of BT columns, then SC code
-// stages of 64 columns (256 k).
-template <int BT, int SA, int SC, int SP, int SK>
+// abort flag.  Tensor memory: NACC accumulators of BT columns (two let a
+// unit's epilogue overlap the next unit's main loop; one leaves room for more
+// code stages), then SC code stages of SK / 4 columns.
+template <int BT, int SA, int SC, int SP, int SK, int NACC = 2>
 struct TcSmem {
     static_assert(SK == 256 || SK == 512, "k per stage");
     static constexpr int kABoxes = SK / kTcBK;                   // activation boxes per stage
@@ -99,9 +151,10 @@ struct TcSmem {
     static constexpr int kBarCount = 2 * SA + 2 * SP + 2 * SC + 5;
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kBytes = kMisc + 16;
-    static constexpr int kCodeCol = 2 * BT;                      // first code-stage column
+    static_assert(NACC == 1 || NACC == 2, "accumulators");
+    static constexpr int kCodeCol = NACC * BT;                   // first code-stage column
     static constexpr int kCodeCols = SK / 4;                     // 32-bit columns of one code stage
-    static constexpr int kTmemNeed = 2 * BT + kCodeCols * SC;
+    static constexpr int kTmemNeed = NACC * BT + kCodeCols * SC;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "tensor memory");
@@ -230,11 +283,11 @@ __device__ __forceinline__ TcUnit tc_unit(const GemmTcArgs &a, int u) {
     return t;
 }
 
-template <int BT, bool BF16_OUT, int SA, int SC, int SP, int SK>
+template <int BT, bool BF16_OUT, int SA, int SC, int SP, int SK, int NACC = 2>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_w2a8_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap pmap,
                         const __grid_constant__ CUtensorMap ymap, const GemmTcArgs a) {
-    using L = TcSmem<BT, SA, SC, SP, SK>;
+    using L = TcSmem<BT, SA, SC, SP, SK, NACC>;
     static_assert(BT % 16 == 0 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -293,6 +346,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     pdl_launch_dependents();
 
+    if (a.x != nullptr && warp >= 2) {
+        // quantisation phase (warps 2..13, one token row per warp at a time,
+        // rows dealt over all CTAs); the weights the producer requested above
+        // land meanwhile.  x may come from the previous kernel and q / s may
+        // still be read by it: wait for it first.
+        pdl_wait();
+        constexpr int kQWarps = kTcThreads / 32 - 2;
+        uint32_t rows = 0;
+        for (int64_t m = (int64_t)blockIdx.x * kQWarps + (warp - 2); m < a.M; m += (int64_t)gridDim.x * kQWarps) {
+            int sum = 0;
+            const float sc = quant_row<1>(a.x + m * a.K, a.K, a.qout + m * a.ldq, a.ldq, true, false, sum, nullptr,
+                                          nullptr, 0, lane);
+            if (lane == 0) const_cast<float *>(a.s_act)[m] = sc;
+            ++rows;
+        }
+        // every lane's rows visible at gpu scope (and to the async proxy) before the count
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0 && rows > 0) tagged_add(&a.sync[0], a.epoch, rows);
+    }
+
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
@@ -314,6 +389,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // weights never depend on an earlier kernel; activations may
             while (up < units && ip < SP) issue_p();
             pdl_wait();
+            // quantisation inside this launch: every row of q (written by the
+            // generic proxy of all CTAs) is in place before the first TMA read
+            bool q_ready = true;
+            if (a.x != nullptr) {
+                q_ready = wait_tagged(&a.sync[0], a.epoch, (uint32_t)a.M, abort_flag);
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            if (!q_ready) ua = up = units;  // aborted: issue nothing more
             // poll both rings without blocking on either (a blocking wait on one
             // would hold back the other); the idle time is bounded like every wait
             uint64_t idle_since = 0;
@@ -367,9 +450,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int g = 0;  // stages consumed over all units
             int li = 0;
             for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++li) {
-                const int d = li & 1;
+                const int d = li % NACC;
                 // the epilogue has drained this accumulator's previous unit
-                if (li >= 2 && !tc_wait(&accum_empty[d], (uint32_t)((li >> 1) - 1) & 1u, abort_flag)) {
+                if (li >= NACC && !tc_wait(&accum_empty[d], (uint32_t)((li / NACC) - 1) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -471,11 +554,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int nbox = 0;  // boxes this warp has stored (its staging buffers take turns)
         int li = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++li) {
-            const int d = li & 1;
-            if (!tc_wait(&accum_full[d], (uint32_t)(li >> 1) & 1u, abort_flag)) break;
+            const int d = li % NACC;
+            if (!tc_wait(&accum_full[d], (uint32_t)(li / NACC) & 1u, abort_flag)) break;
             tc_fence_after();
             if (!waited_pdl) {
                 pdl_wait();  // the outputs may still be read by the previous kernel
+                // scales written in this launch by other CTAs: complete (the
+                // MMAs waited for every row) and acquired here before use
+                if (a.x != nullptr && !wait_tagged(&a.sync[0], a.epoch, (uint32_t)a.M, abort_flag)) break;
                 waited_pdl = true;
             }
             const TcUnit t = tc_unit(a, u);
@@ -557,6 +643,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::kTmemCols)
                      : "memory");
+    }
+    // the last CTA to finish returns the counters to {epoch, 0}: nothing of
+    // this launch reads them any more
+    if (a.x != nullptr && threadIdx.x == 0 && tagged_add(&a.sync[1], a.epoch, 1) == gridDim.x) {
+        const unsigned long long z = (unsigned long long)a.epoch << 32;
+        atomicExch(&a.sync[0], z);
+        atomicExch(&a.sync[1], z);
     }
 }
 

@@ -93,7 +93,7 @@ __device__ __forceinline__ void stage_q_int8(uint4 *qs, const int8_t *qrow, int6
     }
 }
 
-// Fused per-token quantisation (same arithmetic as quant_act_kernel): absmax
+// Fused per-token quantisation (same arithmetic as quant_act_kernel<>): absmax
 // over the whole row, then the slice's codes into qs.  Returns the scale.
 // Thread t owns the 16-value pieces t, t + blockDim, ...; up to kHeld of them
 // stay in registers between the absmax pass and the quantise pass.

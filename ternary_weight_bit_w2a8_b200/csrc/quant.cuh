@@ -21,64 +21,151 @@ __device__ __forceinline__ int8_t quant_one(float x, float sc) {
     return (int8_t)r;
 }
 
-// One CTA per token.  Writes q with row stride ldq (>= K); positions
-// K <= k < ldq are written as 0 when zero_pad is set.
-__global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t *__restrict__ x, int64_t K,
-                                                             int8_t *__restrict__ q, int64_t ldq,
-                                                             bool zero_pad, float *__restrict__ s,
-                                                             int32_t *__restrict__ rowsum) {
-    __shared__ float fscratch[32];
-    __shared__ int iscratch[32];
-    // a dependent kernel may start its own independent work (weight loads) now;
-    // it waits for this grid to complete before it reads q or s
-    pdl_launch_dependents();
-    const int64_t m = blockIdx.x;
-    const uint16_t *xr = x + m * K;
-    int8_t *qr = q + m * ldq;
-    const bool vec = ((reinterpret_cast<uintptr_t>(xr) & 15) == 0);
-    const int64_t K8 = vec ? (K / 8) * 8 : 0;
-    const bool qvec = vec && ((reinterpret_cast<uintptr_t>(qr) & 7) == 0);
+// |x| maximum over the 8 bf16 values of a 16-byte word.
+__device__ __forceinline__ float amax8(const uint4 &v, float m) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m = fmaxf(m, fabsf(__uint_as_float(w[i] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(w[i] & 0xffff0000u)));
+    }
+    return m;
+}
 
+// The 8 codes of a 16-byte word of bf16 values (low byte = lowest k), and
+// their sum added to `sum`.
+__device__ __forceinline__ uint2 quant8(const uint4 &v, float sc, int &sum) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int8_t lo = quant_one(__uint_as_float(w[i] << 16), sc);
+        const int8_t hi = quant_one(__uint_as_float(w[i] & 0xffff0000u), sc);
+        sum += lo + hi;
+        o[i >> 1] |= ((uint32_t)(uint8_t)lo | ((uint32_t)(uint8_t)hi << 8)) << (16 * (i & 1));
+    }
+    return make_uint2(o[0], o[1]);
+}
+
+// A team of WPT warps quantises one token row at a time (a CTA of kThreads
+// threads holds kThreads / (32 * WPT) teams; rows are dealt to teams
+// grid-stride).  The row is read from HBM once: each thread keeps up to
+// kQuantHeld 16-byte words in registers between the absmax pass and the
+// quantise pass (rows longer than kQuantHeld * 8 * 32 * WPT values re-read
+// the rest, from L1/L2).  Reductions are warp shuffles plus, for WPT > 1, one
+// named barrier per team.  q rows have stride ldq (>= K); with zero_pad set,
+// K <= k < ldq is written as 0.  rowsum may be null.
+constexpr int kQuantHeld = 12;
+
+template <int WPT>
+__device__ __forceinline__ float team_max(float v, float *red, int team, int wt) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (WPT > 1) {
+        if ((threadIdx.x & 31) == 0) red[team * WPT + wt] = v;
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(WPT * 32) : "memory");
+        v = red[team * WPT];
+#pragma unroll
+        for (int i = 1; i < WPT; ++i) v = fmaxf(v, red[team * WPT + i]);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(WPT * 32) : "memory");
+    }
+    return v;
+}
+
+template <int WPT>
+__device__ __forceinline__ int team_sum(int v, int *red, int team, int wt) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (WPT > 1) {
+        if ((threadIdx.x & 31) == 0) red[team * WPT + wt] = v;
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(WPT * 32) : "memory");
+        int r = 0;
+#pragma unroll
+        for (int i = 0; i < WPT; ++i) r += red[team * WPT + i];
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(WPT * 32) : "memory");
+        v = r;
+    }
+    return v;
+}
+
+// One token row quantised by a team of WPT warps (team-local thread t of
+// 32 * WPT; `team` picks the named barrier and the reduction slots).  Writes
+// q (and the zero padding up to ldq), returns the scale; `sum` receives the
+// row's code sum when want_sum is set.
+template <int WPT>
+__device__ __forceinline__ float quant_row(const uint16_t *__restrict__ xr, int64_t K, int8_t *__restrict__ qr,
+                                           int64_t ldq, bool zero_pad, bool want_sum, int &sum, float *fred,
+                                           int *ired, int team, int t) {
+    constexpr int kTeam = 32 * WPT;
+    const int wt = t >> 5;
+    const bool vec = (reinterpret_cast<uintptr_t>(xr) & 15) == 0;
+    const bool qvec = (reinterpret_cast<uintptr_t>(qr) & 7) == 0;
+    const int64_t nw = vec ? K / 8 : 0;  // whole 16-byte words of the row
+
+    uint4 held[kQuantHeld];
     float amax = 0.0f;
-    for (int64_t k = threadIdx.x * 8; k < K8; k += kThreads * 8) {
-        uint4 v = *reinterpret_cast<const uint4 *>(xr + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xffff0000u)));
+    for (int i = 0; i < kQuantHeld; ++i) {
+        const int64_t c = t + (int64_t)i * kTeam;
+        if (c < nw) {
+            held[i] = *reinterpret_cast<const uint4 *>(xr + 8 * c);
+            amax = amax8(held[i], amax);
         }
     }
-    for (int64_t k = K8 + threadIdx.x; k < K; k += kThreads) amax = fmaxf(amax, fabsf(bf16_bits_to_float(xr[k])));
-    amax = block_reduce(amax, [](float a, float b) { return fmaxf(a, b); }, fscratch);
-
+    for (int64_t c = t + (int64_t)kQuantHeld * kTeam; c < nw; c += kTeam)
+        amax = amax8(*reinterpret_cast<const uint4 *>(xr + 8 * c), amax);
+    for (int64_t k = nw * 8 + t; k < K; k += kTeam) amax = fmaxf(amax, fabsf(bf16_bits_to_float(xr[k])));
+    amax = team_max<WPT>(amax, fred, team, wt);
     const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
-    int sum = 0;
-    const int64_t Kv = qvec ? K8 : 0;  // 8 values per thread: one 16-byte load, one 8-byte store
-    for (int64_t k = threadIdx.x * 8; k < Kv; k += kThreads * 8) {
-        uint4 v = *reinterpret_cast<const uint4 *>(xr + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t packed[2] = {0u, 0u};
+
+    sum = 0;
+    auto put8 = [&](int64_t c, const uint2 &v) {
+        if (qvec) {
+            *reinterpret_cast<uint2 *>(qr + 8 * c) = v;
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int8_t lo = quant_one(__uint_as_float(w[i] << 16), sc);
-            const int8_t hi = quant_one(__uint_as_float(w[i] & 0xffff0000u), sc);
-            sum += lo + hi;
-            packed[i >> 1] |= ((uint32_t)(uint8_t)lo | ((uint32_t)(uint8_t)hi << 8)) << (16 * (i & 1));
+            for (int b = 0; b < 8; ++b) qr[8 * c + b] = (int8_t)(((b < 4 ? v.x : v.y) >> (8 * (b & 3))) & 0xff);
         }
-        *reinterpret_cast<uint2 *>(qr + k) = make_uint2(packed[0], packed[1]);
+    };
+#pragma unroll
+    for (int i = 0; i < kQuantHeld; ++i) {
+        const int64_t c = t + (int64_t)i * kTeam;
+        if (c < nw) put8(c, quant8(held[i], sc, sum));
     }
-    for (int64_t k = Kv + threadIdx.x; k < K; k += kThreads) {
+    for (int64_t c = t + (int64_t)kQuantHeld * kTeam; c < nw; c += kTeam)
+        put8(c, quant8(*reinterpret_cast<const uint4 *>(xr + 8 * c), sc, sum));
+    for (int64_t k = nw * 8 + t; k < K; k += kTeam) {
         const int8_t qi = quant_one(bf16_bits_to_float(xr[k]), sc);
         qr[k] = qi;
         sum += qi;
     }
     if (zero_pad)
-        for (int64_t k = K + threadIdx.x; k < ldq; k += kThreads) qr[k] = 0;
-    sum = block_reduce(sum, [](int a, int b) { return a + b; }, iscratch);
-    if (threadIdx.x == 0) {
-        s[m] = sc;
-        if (rowsum != nullptr) rowsum[m] = sum;
+        for (int64_t k = K + t; k < ldq; k += kTeam) qr[k] = 0;
+    if (want_sum) sum = team_sum<WPT>(sum, ired, team, wt);
+    return sc;
+}
+
+template <int WPT>
+__global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                             int8_t *__restrict__ q, int64_t ldq, bool zero_pad,
+                                                             float *__restrict__ s, int32_t *__restrict__ rowsum) {
+    constexpr int kTeam = 32 * WPT;
+    constexpr int kTeams = kThreads / kTeam;
+    __shared__ float fred[kThreads / 32];
+    __shared__ int ired[kThreads / 32];
+    // a dependent kernel may start its own independent work (weight loads)
+    // now; it waits for this grid to complete before it reads q or s
+    pdl_launch_dependents();
+    pdl_wait();
+    const int team = threadIdx.x / kTeam, t = threadIdx.x % kTeam;
+    for (int64_t m = (int64_t)blockIdx.x * kTeams + team; m < M; m += (int64_t)gridDim.x * kTeams) {
+        int sum = 0;
+        const float sc = quant_row<WPT>(x + m * K, K, q + m * ldq, ldq, zero_pad, rowsum != nullptr, sum, fred, ired,
+                                        team, t);
+        if (t == 0) {
+            s[m] = sc;
+            if (rowsum != nullptr) rowsum[m] = sum;
+        }
     }
 }
 

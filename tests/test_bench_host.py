@@ -87,13 +87,13 @@ def test_reference_arm_other_ranks_exit_quietly():
 
 def test_traffic_valid_only_for_the_captured_sources(tmp_path):
     h = bench.kernel_source_hash()
-    good = tmp_path / "t.md"
-    good.write_text(f"notes: x\nsource_sha256: `{h}`\ntraffic_bytes_per_launch: `1234.5`\n")
+    good = tmp_path / "t.json"
+    good.write_text(json.dumps({"source_sha256": h, "traffic_bytes_per_launch": 1234.5}))
     assert bench.read_traffic(str(good)) == 1234.5
-    stale = tmp_path / "s.md"
-    stale.write_text("source_sha256: `" + "0" * 64 + "`\ntraffic_bytes_per_launch: `1234.5`\n")
+    stale = tmp_path / "s.json"
+    stale.write_text(json.dumps({"source_sha256": "0" * 64, "traffic_bytes_per_launch": 1234.5}))
     assert bench.read_traffic(str(stale)) is None
-    assert bench.read_traffic(str(tmp_path / "missing.md")) is None
+    assert bench.read_traffic(str(tmp_path / "missing.json")) is None
 
 
 def test_replay_steps_runs_exactly_n_steps():

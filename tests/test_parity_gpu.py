@@ -48,6 +48,7 @@ def bf16_tensor(bits):
 def check_bf16(y_gpu, y_ref):
     """max relative error 1e-2, absolute 1e-3 where |y_ref| < 0.1."""
     y = y_gpu.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(y).all(), "non-finite bf16 output"
     err = np.abs(y - y_ref)
     near = np.abs(y_ref) < 0.1
     bad = np.where(near, err > 1e-3, err > 1e-2 * np.abs(y_ref))
@@ -152,6 +153,53 @@ def test_gemv_extreme_values():
     assert y.tolist() == [[-128 * K] * 3]
 
 
+# The TMA-staged GEMV keeps one row's whole K on one lane: |acc_j| <= 4096 K per
+# lane is exact for K <= 2^19, and its shared-memory plan caps K well below
+# that.  Forced to its smallest ring (4 warps x 1 box: the most room for the
+# activations), it takes K = 208896 in one CTA; all weights +1 (code 2, the
+# largest scaled code) against activations of -128 is the extreme there.
+TMA_MAX_K_CHILD = r"""
+import json, sys
+import numpy as np, torch
+sys.path.insert(0, ROOT)
+import ternary_weight_bit_w2a8_b200 as bn
+out = {}
+for (N, K) in [(32, 208896), (5, 163840), (64, 131072)]:
+    w = np.ones((N, K), np.int8)
+    packed = bn.bitnet_pack_weights(torch.from_numpy(w).cuda())
+    for val in (-128, 127):
+        q = np.full((1, K), val, np.int8)
+        y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), packed, N).cpu().numpy()
+        out[f"{N}x{K}x{val}"] = bool((y == val * K).all())
+    w[:, 1::2] = -1
+    q = np.full((1, K), -128, np.int8)
+    y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), bn.bitnet_pack_weights(torch.from_numpy(w).cuda()),
+                            N).cpu().numpy()
+    out[f"{N}x{K} alternating"] = bool((y == 0).all())
+torch.cuda.synchronize()
+out["device_error"] = bn.bitnet_get_device_error()
+out["launches"] = bn.bitnet_launch_count()
+print(json.dumps(out))
+"""
+
+
+def test_gemv_tma_largest_k_extremes():
+    import json
+    import os
+    import subprocess
+    import sys
+    from conftest import ROOT
+    env = dict(os.environ)
+    env["BITNET_GEMV_TUNE"] = "0,0,0,0,-1,0,-1,1,0,4"  # TMA GEMV, 4 warps, ring of one box
+    r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + TMA_MAX_K_CHILD], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert res.pop("device_error") == 0
+    assert res.pop("launches") > 0
+    assert all(res.values()), res
+
+
 @pytest.mark.parametrize("N,K", [(64, 65536), (3, 100000), (200, 200000)])
 def test_gemv_split_k_exact(N, K):
     q, w, y = gemv_case(N, K, seed=K)
@@ -232,21 +280,28 @@ def test_gemm_small_batch_exact(M, N, K):
 @pytest.mark.parametrize("M", synth.PREFILL_M)
 @pytest.mark.parametrize("N,K", synth.PREFILL_SHAPES)
 def test_prefill_int32_and_bf16(M, N, K):
-    x, wt, g, packed, y = bitlinear_case(M, N, K, seed=0, outliers=False)
+    """Production-size prefill, every output element: int32 bit-exact against
+    the oracle's full contraction, bf16 within the stated tolerance of its fp64
+    rescale; outputs and workspaces sit between guard bands."""
+    from guarded import Guarded, guarded_workspace
+    x, W = synth.bitlinear_inputs(M, N, K, seed=0, outliers=False)
+    g = oracle.absmean(W)
+    wt = oracle.ternarize(W, g)
+    packed = pack_on_gpu(wt)
     q, s, _ = bn.bitnet_quant_act(bf16_tensor(x))
     q_ref, s_ref, _ = oracle.quant_act(x)
     assert np.array_equal(host(q), q_ref)
-    acc = host(bn.bitnet_w2a8_gemm(q, packed, N))
-    rng = np.random.default_rng(M)
-    if M <= 128:
-        acc_ref = oracle.gemm_i32(q_ref, wt)
-        assert np.array_equal(acc, acc_ref)
-        y_ref = oracle.rescale(acc_ref, g, s_ref)
-        check_bf16(y, y_ref)
-    else:
-        ms = rng.integers(0, M, 4096)
-        ns = rng.integers(0, N, 4096)
-        ref = oracle.gemm_i32_sampled(q_ref, wt, ms, ns)
-        assert np.array_equal(acc[ms, ns], ref)
-        y_ref = oracle.rescale(ref.reshape(-1, 1), g, s_ref[ms])
-        check_bf16(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()].reshape(-1, 1), y_ref)
+    yg = Guarded(torch, (M, N), torch.int32, fill=-7)
+    wsg = guarded_workspace(torch, bn, M, N, K)
+    bn.bitnet_w2a8_gemm(q, packed, N, y=yg.t, ws=wsg.t)
+    acc_ref = oracle.gemm_i32(q_ref, wt)
+    assert np.array_equal(host(yg.t), acc_ref)
+    yg.check("the int32 output")
+    wsg.check("the workspace")
+    bg = Guarded(torch, (M, N), torch.int16, fill=0x7F7F)
+    wsb = guarded_workspace(torch, bn, M, N, K)
+    bn.bitnet_bitlinear(bf16_tensor(x), packed, dev(np.array([g], np.float32)), N,
+                        y=bg.t.view(torch.bfloat16), ws=wsb.t)
+    check_bf16(bg.t.view(torch.bfloat16), oracle.rescale(acc_ref, g, s_ref))
+    bg.check("the bf16 output")
+    wsb.check("the BitLinear workspace")

@@ -49,3 +49,29 @@ def test_small_batch_bitlinear(M, N, K):
     err = np.abs(yf - y_ref)
     assert np.where(np.abs(y_ref) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(y_ref)).all()
     assert not y.view(torch.int16).cpu().numpy()[1].any()
+
+
+def test_bitlinear_same_bits_on_every_path():
+    """A token's bf16 output does not depend on which path quantised it: the
+    single-token prologue (1 token), the multi-token prologue (2..4), a
+    quantisation pass before the GEMV (5..8) or before the tensor-core GEMM (9
+    and more).  All of them take the scale and the codes with the same fp32
+    operations and rescale the same way, so the shared tokens' outputs must be
+    identical bit for bit (a one-ulp scale difference would change codes)."""
+    N, K = 300, 2560
+    x, W = synth.bitlinear_inputs(12, N, K, seed=5)
+    x[7, :] = 0
+    g = oracle.absmean(W)
+    wt = oracle.ternarize(W, g)
+    packed = bn.bitnet_pack_weights(torch.from_numpy(wt).cuda())
+    gamma = torch.tensor([float(g)], dtype=torch.float32, device="cuda")
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    outs = {M: bn.bitnet_bitlinear(xd[:M].contiguous(), packed, gamma, N).view(torch.int16).cpu().numpy()
+            for M in (1, 2, 3, 4, 5, 8, 9, 12)}
+    full = outs[12]
+    for M, y in outs.items():
+        assert np.array_equal(y, full[:M]), f"{M} tokens: bf16 bits differ from the 12-token run"
+    y_ref = oracle.bitlinear(x, wt, g)[0]
+    yf = torch.from_numpy(full).view(torch.bfloat16).float().numpy().astype(np.float64)
+    err = np.abs(yf - y_ref)
+    assert np.where(np.abs(y_ref) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(y_ref)).all()

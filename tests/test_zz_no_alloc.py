@@ -3,8 +3,8 @@
 It serves callers that cannot allocate device memory and therefore cannot pass
 the workspace bitnet_w2a8_gemm may need; it uses the library's one built-in
 scratch array instead.  These tests call it through the C ABI and check it
-against the workspace entry point on the same inputs, two calls in a row with
-different data (the shared scratch keeps the previous call's contents, so a
+against the oracle and against the workspace entry point on the same inputs,
+two calls in a row with different data (the shared scratch keeps the previous call's contents, so a
 stale read would show), including a shape whose plan does use scratch.  This
 file is collected last on purpose.
 """
@@ -13,6 +13,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 import ternary_weight_bit_w2a8_b200 as bn
 from ternary_weight_bit_w2a8_b200 import synth
 
@@ -56,5 +57,6 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
                                               ctypes.c_void_p(y.data_ptr()), M, N, K, stream)
             assert rc == bn.BITNET_OK, bn.status_string(rc)
             torch.cuda.synchronize()
+            assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w)), (M, N, K, call)
             assert torch.equal(y, y_ref), (M, N, K, call)
     assert bn.bitnet_get_device_error() == 0
