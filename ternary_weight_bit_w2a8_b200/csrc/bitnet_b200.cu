@@ -37,7 +37,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[32] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    size_t tma_max_dyn[22] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[2 * 10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -105,14 +105,6 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// ------------------------------------------------------------------ per-call tags
-// Kernels whose CTAs meet through counters or flags in the workspace tag
-// them with a per-call value, so that no zeroing is needed (see gemv_tma.cuh
-// and gemm_tc.cuh).  The top nibble 0xA keeps every tag outside the range of
-// the int32 partial sums (|sum| < 2^28) that share the workspace.
-std::atomic<uint32_t> g_epoch{1};
-inline uint32_t next_epoch() { return 0xA0000000u | (g_epoch.fetch_add(1, std::memory_order_relaxed) & 0x0FFFFFFFu); }
-
 // ------------------------------------------------------------------ activation quantisation
 // Teams of 1..8 warps per token: about a thousand warps in flight whatever M
 // (one warp per token from 1024 tokens up), so the pass is one wave that reads
@@ -149,12 +141,13 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
-// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,split,warps,fuse"
-// (register GEMV: G, R, U, ctas, prefetch, S; tensor-core GEMM: R < 0 token
-// tile, S K-splits, fuse = 0 quantises BitLinear activations in a pass of
-// their own; TMA GEMV: tma = 0 off, ns ring depth, split -1/0/1, warps)
+// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse"
+// (register GEMV: G, R, U, ctas, prefetch, S; TMA GEMV: tma = 0 off or
+// 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth; tensor-core GEMM:
+// R < 0 variant, S K-splits, fuse = 1 quantises BitLinear activations inside
+// the GEMM launch)
 struct GemvTune {
-    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, split = -1, warps = 0, fuse = -1;
+    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -163,8 +156,8 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma,
-                   &t.ns, &t.split, &t.warps, &t.fuse);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma, &t.ns,
+                   &t.fuse);
     });
     return t;
 }
@@ -296,49 +289,53 @@ bool encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *ptr, uin
     return true;
 }
 
+// TMA GEMV variants: (warps per CTA, most boxes in flight per warp); the
+// ring depth of a launch is the smaller of the latter and what its items need
+constexpr int kTmaNumCfg = 5;
+constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
 // BitLinear with up to this many tokens quantises them inside the GEMV's
 // prologue (every CTA reads and quantises all of them); more tokens are
-// quantised once by the quantisation pass first.  Measured on B200, 2560 x 6912:
+// quantised once by quant_act_kernel first.  Measured on B200, 2560 x 6912:
 // 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
 constexpr int kFusedQuantMaxTokens = 4;
 
-// Kernel of (mode, warps, tokens per launch): 4, 8, 12 or 16 warps for one or
-// two tokens, 4 or 8 warps for four or eight (the registers of two CTAs per
-// SM), int8 activations (xmode 0) or, up to kFusedQuantMaxTokens tokens, bf16
-// activations quantised in the kernel (xmode 1).  Index in the kernel and
-// shared-memory opt-in tables, -1 if there is no such kernel.
-int tma_kernel_slot(int xmode, int W, int mt) {
-    const int wi = W == 4 ? 0 : (W == 8 ? 1 : (W == 12 ? 2 : (W == 16 ? 3 : -1)));
-    const int mi = mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : (mt == 8 ? 3 : -1)));
-    if (wi < 0 || mi < 0 || (mt >= 4 && W > 8) || (xmode == 1 && mt > kFusedQuantMaxTokens)) return -1;
-    return xmode * 16 + mi * 4 + wi;
+// Kernel of (mode, warps, tokens per launch): one token on 4, 8, 12 or 16
+// warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8 activations
+// (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16 activations
+// quantised in the kernel (xmode 1).  Slot in the shared-memory opt-in table:
+// MT == 1 ? xmode * 10 + W / 4 - 1 : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16);
+// -1 if none.
+int tma_kernel_slot(int xmode, int cfg, int mt) {
+    const int W = kTmaCfg[cfg][0];
+    if (mt == 1) return xmode * 10 + W / 4 - 1;
+    if (W != 8 && W != 16) return -1;
+    if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
+    return xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
 }
 
-TmaKernel tma_kernel_for(int xmode, int W, int mt) {
-    static const TmaKernel table[32] = {
+TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
+    static const TmaKernel table[20] = {
         gemv_tma_kernel<0, 4, 1>, gemv_tma_kernel<0, 8, 1>, gemv_tma_kernel<0, 12, 1>, gemv_tma_kernel<0, 16, 1>,
-        gemv_tma_kernel<0, 4, 2>, gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 12, 2>, gemv_tma_kernel<0, 16, 2>,
-        gemv_tma_kernel<0, 4, 4>, gemv_tma_kernel<0, 8, 4>, nullptr, nullptr,
-        gemv_tma_kernel<0, 4, 8>, gemv_tma_kernel<0, 8, 8>, nullptr, nullptr,
+        gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 16, 4>,
+        gemv_tma_kernel<0, 8, 8>, gemv_tma_kernel<0, 16, 8>,
         gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>,
-        gemv_tma_kernel<1, 4, 2>, gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 12, 2>, gemv_tma_kernel<1, 16, 2>,
-        gemv_tma_kernel<1, 4, 4>, gemv_tma_kernel<1, 8, 4>, nullptr, nullptr,
-        nullptr, nullptr, nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
-    const int slot = tma_kernel_slot(xmode, W, mt);
+        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 16, 2>, gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 16, 4>,
+        nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
+    const int slot = tma_kernel_slot(xmode, cfg, mt);
     return slot < 0 ? nullptr : table[slot];
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int W, int mt) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    const int si = tma_kernel_slot(xmode, W, mt);
+    const int si = tma_kernel_slot(xmode, cfg, mt);
     if (si < 0) return 0;
     size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, W, mt);
+        TmaKernel kern = tma_kernel_for(xmode, cfg, mt);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -349,73 +346,65 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int W, int mt) {
 }
 
 // Plan of the TMA GEMV, from the shape and B200 reference figures only (148
-// SMs, 228 KB of shared memory per SM), so that what a shape needs does not
+// SMs, 227 KB of shared memory per CTA), so that what a shape needs does not
 // depend on the device that runs it.
-//   - One CTA per SM (grid = min(items, 148)).  A CTA takes under half an SM
-//     (registers by the kernel's launch bounds, shared memory here), so the
-//     next launch's CTA is resident beside it and requests its weights while
-//     this launch finishes (programmatic dependent launch).
-//   - Whole row blocks per CTA, or, where that leaves the busiest SM more
-//     than kTmaSplitGainItems items above an even share, an even split of
-//     all (row block, K-slice) items: a row block then spans CTAs, whose
-//     int32 partial sums meet in the workspace (see gemv_tma.cuh).
-//   - Warps and ring depth: the most boxes in flight that leave room for a
-//     second CTA; 16 warps when each takes at most one box, else 12 (8 for
-//     four and eight tokens).
-constexpr int kTmaSplitGainItems = 8;
-
 struct TmaPlan {
     bool use;
-    int W, ns, mt, grid, split, slices, max_slots;
-    int64_t nblocks;
+    int cfg, slices, max_blocks, grid;
+    int ns;            // ring depth per warp
+    int mt;            // tokens per launch (1, 2, 4, 8)
     size_t smem;
-    int64_t ws_bytes;  // split: partial-sum records and their flags
+    int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
 };
 
 TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
-    constexpr size_t kRefSmemOptin = 232448;  // one CTA per SM
-    constexpr size_t kRefSmemHalf = 114688;   // two CTAs per SM (1 KB reserved and static memory each)
-    const GemvTune &tn = gemv_tune();
+    constexpr size_t kRefSmemOptin = 232448;
     TmaPlan p{};
-    if (M < 1 || M > 8 || tn.tma == 0 || K < kTmaSliceK || N < 1) return p;
+    const int tune = gemv_tune().tma;
+    if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
     // a lane accumulates one row's whole K: |acc_j| <= 4096 * K_pad stays
     // inside int32 for K_pad <= 2^19 (shared memory caps K lower still)
     if (k_pad(K) > ((int64_t)1 << 19)) return p;
     p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
-    p.nblocks = ceil_div(N, kTmaRows);
-    p.slices = (int)ceil_div(packed_row_bytes(K), kTmaSliceBytes);
-    const int64_t items = p.nblocks * p.slices;
-    p.grid = (int)(items < kRefSMs ? items : kRefSMs);
-    const int64_t whole = ceil_div(p.nblocks, p.grid) * p.slices;
-    const int64_t even = ceil_div(items, p.grid);
-    p.split = (whole - even > kTmaSplitGainItems) ? 1 : 0;
-    if (tn.split >= 0) p.split = tn.split;
-    const int64_t ipc = p.split ? even : whole;  // most items of one CTA
-    p.max_slots = (int)(p.split ? (ipc - 1) / p.slices + 2 : ceil_div(p.nblocks, p.grid));
-    int W = p.mt >= 4 ? 8 : (ipc <= 16 ? 16 : 12);
-    if (tn.warps > 0 && tma_kernel_slot(0, tn.warps, p.mt) >= 0) W = tn.warps;
-    // ring depth: as deep as the items need and two CTAs per SM allow
-    const size_t fixed = gemv_tma_smem_bytes(W, 0, p.slices, p.max_slots, p.mt);
-    int64_t ns = ceil_div(ipc, W);
-    if (ns > 4) ns = 4;
-    while (ns > 1 && fixed + (size_t)W * ns * (kTmaBoxBytes + 8) > kRefSmemHalf) --ns;
-    if (tn.ns > 0) ns = tn.ns;
-    p.ns = (int)ns;
-    p.W = W;
-    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_slots, p.mt);
+    const int64_t row_bytes = packed_row_bytes(K);
+    const int64_t nblocks = ceil_div(N, kTmaRows);
+    p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
+    // variant (measured on B200 over sequences of different shapes, as in a
+    // decode step): 16 x 2, and 12 x 3 for rows of K >= 16384.  Variants that
+    // let two CTAs share an SM win on a shape repeated alone but lose in a
+    // mixed sequence, where the scheduler can then stack two CTAs of one
+    // launch on an SM.
+    if (tune >= 1 && tune <= kTmaNumCfg)
+        p.cfg = tune - 1;
+    else
+        p.cfg = p.slices >= 32 ? 1 : 2;
+    if (p.mt > 1 && kTmaCfg[p.cfg][0] != 8 && kTmaCfg[p.cfg][0] != 16) p.cfg = 2;  // several tokens: 8 or 16 warps
+    const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
+    // at most one CTA per SM per launch (BITNET_GEMV_TUNE's ctas field
+    // overrides): each SM keeps room for a CTA of the next launch, which then
+    // starts and requests its weights while this one finishes
+    const int per_sm = gemv_tune().ctas > 0 ? gemv_tune().ctas : 1;
+    const int64_t gmax = (int64_t)kRefSMs * per_sm;
+    p.grid = (int)(nblocks < gmax ? nblocks : gmax);
+    p.max_blocks = (int)ceil_div(nblocks, p.grid);
+    // ring depth: no more boxes per warp than its items (a small launch then
+    // needs little shared memory and leaves room beside it)
+    const int64_t ipw = ceil_div((int64_t)p.max_blocks * p.slices, W);
+    p.ns = (int)(ipw < NS ? (ipw < 1 ? 1 : ipw) : NS);
+    if (gemv_tune().ns > 0) p.ns = gemv_tune().ns < NS ? gemv_tune().ns : NS;
+    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_blocks, p.mt);
     if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
-    p.ws_bytes = p.split ? round_up((int64_t)p.grid * p.mt * kTmaRows * 4, 256) + round_up((int64_t)p.grid * 4, 256) : 0;
     p.use = true;
     return p;
 }
 
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
-                    const TmaPlan &tp, void *ws, cudaStream_t st) {
-    TmaKernel kern = tma_kernel_for(xmode, tp.W, tp.mt);
+                    const TmaPlan &tp, cudaStream_t st) {
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
     if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
-    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.W, tp.mt))
+    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
@@ -439,23 +428,16 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.N = N;
     a.K = K;
     a.slices = tp.slices;
-    a.nblocks = tp.nblocks;
-    a.split = tp.split;
-    a.max_slots = tp.max_slots;
+    a.blk_begin = 0;
+    a.nblocks = ceil_div(N, kTmaRows);
+    a.max_blocks_cta = tp.max_blocks;
     a.ns = tp.ns;
     a.y_i32 = y_i32;
     a.y_bf16 = y_bf16;
     a.gamma = gamma;
     a.s_act = s_act;
-    if (tp.split) {
-        a.rec = static_cast<int32_t *>(ws);
-        a.flags = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) +
-                                               round_up((int64_t)tp.grid * tp.mt * kTmaRows * 4, 256));
-        // a tag no int32 partial sum of this library reaches (|sum| < 2^28)
-        a.epoch = next_epoch();
-    }
     a.test_stall = test_stall;
-    return launched(launch_pdl(kern, dim3(tp.grid), dim3(tp.W * 32), tp.smem, st, map, a));
+    return launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
 }
 
 // xmode 0: int8 activations q (row stride ldq); xmode 1: bf16 activations x,
@@ -466,7 +448,7 @@ int launch_gemv(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, 
     {
         const TmaPlan tp = tma_plan(M, N, K);
         if (tp.use && ldq == K)
-            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, ws, st);
+            return launch_gemv_tma(dev, xmode, q, x, packed, M, N, K, y_i32, y_bf16, gamma, s_act, tp, st);
     }
     const GemvSplit sp = plan_split(M, N, K);
     const GemvTune &tn = gemv_tune();
@@ -660,11 +642,11 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
 
 // reduce: add int32 results into y_i32 (which the caller has zeroed).
 // BitLinear with the activation quantisation inside the GEMM launch: the bf16
-// activations and the call's counter words (16 bytes of workspace).
+// activations (the quantised rows go where the activation map points).
 struct TcFuse {
     const uint16_t *x = nullptr;
-    unsigned long long *sync = nullptr;
 };
+std::atomic<uint32_t> g_bar_slot{0};
 
 int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t *packed, int64_t M, int64_t N,
                    int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *s_act, const float *gamma,
@@ -728,8 +710,7 @@ int launch_gemm_tc(DeviceInfo *dev, const int8_t *q, int64_t lda, const uint8_t 
         a.x = fuse.x;
         a.qout = const_cast<int8_t *>(q);
         a.ldq = lda;
-        a.sync = fuse.sync;
-        a.epoch = next_epoch();
+        a.bar_slot = (int)(g_bar_slot.fetch_add(1, std::memory_order_relaxed) % kGridBarSlots);
     }
     // persistent: one CTA per SM (or fewer, when there are fewer work units)
     const int64_t units = (int64_t)a.tiles_n * a.tiles_m * a.splits;
@@ -793,9 +774,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
         p.tc = tc_plan(M, N, K);
         const int64_t qbytes = round_up(M * k_pad(K), 256);
         if (bitlinear) {
-            // quantised activations, scales, the launch's counter words and,
-            // for a K-split, int32 sums
-            p.ws_bytes = qbytes + round_up(M * 4, 256) + 256 + (p.tc.S > 1 ? round_up(M * N * 4, 256) : 0);
+            // quantised activations, scales and, for a K-split, int32 sums
+            p.ws_bytes = qbytes + round_up(M * 4, 256) + (p.tc.S > 1 ? round_up(M * N * 4, 256) : 0);
         } else {
             p.repack = !q_tma_ok;
             p.ws_bytes = p.repack ? qbytes : 0;
@@ -982,21 +962,23 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
     }
     if (p.path == kPathGemv)  // the tokens are quantised inside the GEMV's prologue: one launch
         return launch_gemv(dev, 1, nullptr, x, K, packed, M, N, K, nullptr, y, nullptr, gamma, workspace, st);
-    // the tensor-core GEMM quantises the rows itself (into K_pad-strided,
-    // zero-padded rows of the workspace) and rescales in its bf16 epilogue
+    // quantise into K_pad-strided, zero-padded rows of the workspace, then the
+    // tensor-core GEMM with the bf16 epilogue.  The quantisation pass is a
+    // launch of its own: measured on B200 it beats quantising inside the GEMM
+    // launch (tuning field `fuse` = 1), whose CTAs must all meet at a grid
+    // barrier before the first activation load.
     const int64_t ldq = k_pad(K);
     int8_t *q = static_cast<int8_t *>(workspace);
     float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * ldq, 256));
     TcFuse fuse;
-    fuse.sync = reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(s) + round_up(M * 4, 256));
-    fuse.x = x;
-    if (gemv_tune().fuse == 0) {  // tuning: a quantisation pass of its own first
-        if ((rc = launch_quant(dev, x, M, K, q, ldq, true, s, nullptr, st)) != BITNET_OK) return rc;
-        fuse.x = nullptr;
+    if (gemv_tune().fuse == 1) {
+        fuse.x = x;
+    } else if ((rc = launch_quant(dev, x, M, K, q, ldq, true, s, nullptr, st)) != BITNET_OK) {
+        return rc;
     }
     if (p.tc.S == 1) return launch_gemm_tc(dev, q, ldq, packed, M, N, K, nullptr, y, s, gamma, p.tc, 0, st, fuse);
     // K-split: int32 sums in the workspace, then the rescale to bf16
-    int32_t *acc = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(fuse.sync) + 256);
+    int32_t *acc = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(s) + round_up(M * 4, 256));
     fill_kernel<int32_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(acc, M * N, 0);
     if ((rc = launched()) != BITNET_OK) return rc;
     if ((rc = launch_gemm_tc(dev, q, ldq, packed, M, N, K, acc, nullptr, s, nullptr, p.tc, 1, st, fuse)) != BITNET_OK)
@@ -1034,6 +1016,9 @@ BITNET_API int bitnet_get_device_error(void *stream) {
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BITNET_ERR_CUDA;
+        // a launch that gave up may have left a grid barrier half-counted
+        static const unsigned int zeros[kGridBarSlots] = {};
+        if (cudaMemcpyToSymbol(g_grid_bar, zeros, sizeof(zeros)) != cudaSuccess) return BITNET_ERR_CUDA;
     }
     return v;
 }

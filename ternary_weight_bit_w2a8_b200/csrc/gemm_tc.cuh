@@ -77,49 +77,49 @@ struct GemmTcArgs {
     const float *s_act;     // [M] activation scales (BitLinear)
     const float *gamma;     // weight scale (BitLinear)
     // BitLinear with the quantisation inside this launch (x != null): bf16
-    // activations x [M, K] are quantised by warps 2..13 of every CTA into
+    // activations x [M, K] are quantised by the epilogue warps of every CTA into
     // qout (rows of ldq bytes, zero-padded: the tensor the activation map
-    // reads) and s_act; sync[0] counts the rows done, sync[1] the CTAs that
-    // finished, both tagged with this call's epoch (see tagged_add)
+    // reads) and s_act; the CTAs then meet at grid barrier `bar_slot` before
+    // the first activation load
     const uint16_t *x;
     int8_t *qout;
     int64_t ldq;
-    unsigned long long *sync;
-    uint32_t epoch;
+    int bar_slot;
 };
 
-// Adds n to a counter word {tag (high 32 bits) : count (low 32 bits)} and
-// returns the new count.  A word whose tag is not `epoch` (left by an earlier
-// call, or never written) counts from zero, so the counter needs no zeroing;
-// the last user of a call resets it to {epoch, 0} so that a replayed CUDA
-// graph (same epoch) starts from zero too.
-__device__ __forceinline__ uint32_t tagged_add(unsigned long long *w, uint32_t epoch, uint32_t n) {
-    unsigned long long cur = atomicAdd(w, 0ull);
-    for (;;) {
-        const uint32_t tag = (uint32_t)(cur >> 32), c = (uint32_t)cur;
-        const unsigned long long nv = ((unsigned long long)epoch << 32) | (unsigned long long)((tag == epoch ? c : 0u) + n);
-        const unsigned long long prev = atomicCAS(w, cur, nv);
-        if (prev == cur) return (uint32_t)nv;
-        cur = prev;
-    }
-}
+// Grid barriers for launches whose CTAs must all finish a phase before any
+// goes on (every CTA of such a launch is resident: one per SM at most).  A
+// barrier is one word in device memory owned by this library (zero at load):
+// each CTA adds 1, CTA 0 adds 2^31 - (G - 1), so the top bit flips exactly
+// when all G have arrived and the low bits return to where they were: the
+// word is ready for its next use with no reset, replayed CUDA graphs
+// included.  Calls take slots in turn, so launches that overlap on the GPU
+// (consecutive calls under programmatic launch) use different words.
+constexpr int kGridBarSlots = 1024;
+__device__ unsigned int g_grid_bar[kGridBarSlots];
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned int ld_acquire_u32g(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
-// Bounded wait until the counter holds {epoch, target}; false after the limit
-// or when another role raised the abort flag.
-__device__ __forceinline__ bool wait_tagged(const unsigned long long *w, uint32_t epoch, uint32_t target,
-                                            volatile int *abort_flag) {
-    const unsigned long long want = ((unsigned long long)epoch << 32) | target;
-    if (ld_acquire_u64(w) == want) return true;
+// Arrival of this CTA (one thread; its CTA's writes made visible before);
+// returns the word as it was before, for grid_bar_wait.
+__device__ __forceinline__ unsigned int grid_bar_arrive(int slot) {
+    __threadfence();
+    const unsigned int inc = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+    return atomicAdd(&g_grid_bar[slot], inc);
+}
+
+// Bounded wait for the flip; false after the limit or when another role
+// raised the abort flag.
+__device__ __forceinline__ bool grid_bar_wait(int slot, unsigned int old, volatile int *abort_flag) {
+    if ((ld_acquire_u32g(&g_grid_bar[slot]) ^ old) & 0x80000000u) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        __nanosleep(64);
-        if (ld_acquire_u64(w) == want) return true;
+        __nanosleep(32);
+        if ((ld_acquire_u32g(&g_grid_bar[slot]) ^ old) & 0x80000000u) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
@@ -346,56 +346,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     pdl_launch_dependents();
 
-    if (a.x != nullptr && warp >= 2) {
-        // quantisation phase (warps 2..13, one token row per warp at a time,
-        // rows dealt over all CTAs); the weights the producer requested above
-        // land meanwhile.  x may come from the previous kernel and q / s may
-        // still be read by it: wait for it first.
+    if (a.x != nullptr && warp >= kTcEpiWarp) {
+        // quantisation phase (the four epilogue warps, idle until the first
+        // accumulator is done: one token row per warp at a time, rows dealt
+        // over all CTAs) while the decoders turn the first packed stages into
+        // codes.  x may come from the previous kernel and q / s may still be
+        // read by it: wait for it first.
         pdl_wait();
-        constexpr int kQWarps = kTcThreads / 32 - 2;
-        uint32_t rows = 0;
-        for (int64_t m = (int64_t)blockIdx.x * kQWarps + (warp - 2); m < a.M; m += (int64_t)gridDim.x * kQWarps) {
+        constexpr int kQWarps = 4;
+        int rows = 0;
+        for (int64_t m = (int64_t)blockIdx.x * kQWarps + (warp - kTcEpiWarp); m < a.M;
+             m += (int64_t)gridDim.x * kQWarps) {
             int sum = 0;
             const float sc = quant_row<1>(a.x + m * a.K, a.K, a.qout + m * a.ldq, a.ldq, true, false, sum, nullptr,
                                           nullptr, 0, lane);
             if (lane == 0) const_cast<float *>(a.s_act)[m] = sc;
             ++rows;
         }
-        // every lane's rows visible at gpu scope (and to the async proxy) before the count
+        (void)rows;
+        // every lane's rows visible at gpu scope (and to the async proxy), then
+        // meet the producer, which arrives at the grid barrier for the CTA
         __threadfence();
         asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-        if (lane == 0 && rows > 0) tagged_add(&a.sync[0], a.epoch, rows);
+        asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");
     }
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            // cursors (unit, stage) of the next activation and packed loads; ia /
-            // ip count the loads issued over all of this CTA's units
-            int ua = blockIdx.x, ka = 0, up = blockIdx.x, kp = 0, ia = 0, ip = 0;
-            TcUnit ta = tc_unit(a, ua), tp = ta;
-            auto issue_p = [&]() {
-                mbar_arrive_expect_tx(&p_full[ip % SP], L::kPStage);
-                tma_load_2d(sm + L::kP + (ip % SP) * L::kPStage, &pmap, (tp.z * a.sps + kp) * L::kPRow, tp.nt * kTcRows,
-                            &p_full[ip % SP]);
-                ++ip;
-                if (++kp == unit_stages(tp)) {
-                    kp = 0;
-                    up += gridDim.x;
-                    if (up < units) tp = tc_unit(a, up);
-                }
-            };
-            // weights never depend on an earlier kernel; activations may
+        // cursors (unit, stage) of the next activation and packed loads; ia /
+        // ip count the loads issued over all of this CTA's units (lane 0 only)
+        int ua = blockIdx.x, ka = 0, up = blockIdx.x, kp = 0, ia = 0, ip = 0;
+        TcUnit ta = tc_unit(a, ua), tp = ta;
+        auto issue_p = [&]() {
+            mbar_arrive_expect_tx(&p_full[ip % SP], L::kPStage);
+            tma_load_2d(sm + L::kP + (ip % SP) * L::kPStage, &pmap, (tp.z * a.sps + kp) * L::kPRow, tp.nt * kTcRows,
+                        &p_full[ip % SP]);
+            ++ip;
+            if (++kp == unit_stages(tp)) {
+                kp = 0;
+                up += gridDim.x;
+                if (up < units) tp = tc_unit(a, up);
+            }
+        };
+        // weights never depend on an earlier kernel; activations may
+        if (lane == 0)
             while (up < units && ip < SP) issue_p();
-            pdl_wait();
-            // quantisation inside this launch: every row of q (written by the
-            // generic proxy of all CTAs) is in place before the first TMA read
-            bool q_ready = true;
-            if (a.x != nullptr) {
-                q_ready = wait_tagged(&a.sync[0], a.epoch, (uint32_t)a.M, abort_flag);
+        // quantisation inside this launch: this CTA's quantisation warps are
+        // done, then every CTA's (grid barrier), so every row of q, written
+        // through the generic proxy, is in place before the first TMA read
+        bool q_ready = true;
+        if (a.x != nullptr) {
+            __syncwarp();
+            asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");  // with the four quantising warps
+            if (lane == 0) {
+                const unsigned int old = grid_bar_arrive(a.bar_slot);
+                q_ready = grid_bar_wait(a.bar_slot, old, abort_flag);
                 asm volatile("fence.proxy.async.global;" ::: "memory");
             }
+        }
+        if (lane == 0) {
+            pdl_wait();
             if (!q_ready) ua = up = units;  // aborted: issue nothing more
             // poll both rings without blocking on either (a blocking wait on one
             // would hold back the other); the idle time is bounded like every wait
@@ -560,8 +570,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!waited_pdl) {
                 pdl_wait();  // the outputs may still be read by the previous kernel
                 // scales written in this launch by other CTAs: complete (the
-                // MMAs waited for every row) and acquired here before use
-                if (a.x != nullptr && !wait_tagged(&a.sync[0], a.epoch, (uint32_t)a.M, abort_flag)) break;
+                // MMAs waited for the grid barrier) and acquired here before use
+                if (a.x != nullptr) (void)ld_acquire_u32g(&g_grid_bar[a.bar_slot]);
                 waited_pdl = true;
             }
             const TcUnit t = tc_unit(a, u);
@@ -643,13 +653,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::kTmemCols)
                      : "memory");
-    }
-    // the last CTA to finish returns the counters to {epoch, 0}: nothing of
-    // this launch reads them any more
-    if (a.x != nullptr && threadIdx.x == 0 && tagged_add(&a.sync[1], a.epoch, 1) == gridDim.x) {
-        const unsigned long long z = (unsigned long long)a.epoch << 32;
-        atomicExch(&a.sync[0], z);
-        atomicExch(&a.sync[1], z);
     }
 }
 

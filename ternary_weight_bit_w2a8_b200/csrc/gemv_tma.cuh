@@ -51,58 +51,24 @@ struct GemvTmaArgs {
     int M;                // tokens of this launch (<= the kernel's MT)
     int64_t N, K;
     int slices;           // K-slices of 128 packed bytes per row
-    int64_t nblocks;      // row blocks of 32 rows
-    int split;            // 1: CTA c owns items [c*I/G, (c+1)*I/G) of the I = nblocks * slices
-                          // items; 0: whole row blocks [c*nblocks/G, (c+1)*nblocks/G)
-    int max_slots;        // accumulator slots (row blocks) per CTA
+    int64_t blk_begin;    // first row block of this launch
+    int64_t nblocks;      // row blocks of this launch
+    int max_blocks_cta;   // accumulator slots per CTA
     int ns;               // ring depth per warp: boxes in flight
     int32_t *y_i32;       // [M, N] int32 result
     uint16_t *y_bf16;     // [M, N] bf16 result (BitLinear)
     const float *gamma;   // weight scale (BitLinear)
     const float *s_act;   // mode 0 with bf16 output: per-token activation scales [M]
-    int32_t *rec;         // split: [G][MT][32] int32 partial sums of each CTA's first row block
-    uint32_t *flags;      // split: [G] record flags (== epoch when the record is valid)
-    uint32_t epoch;       // split: this call's tag (never 0)
     int test_stall;       // test hook: warp 0 never requests its first box, so its first wait times out
 };
 
 // Dynamic shared memory of a launch: ring of warps x stages boxes, linear
 // activations, per-row-block accumulators and counters, slice sums, mbarriers.
-__host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_slots,
+__host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta,
                                                       int tokens = 1) {
     return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes +
-           (size_t)tokens * slices * kTmaSliceK + (size_t)max_slots * tokens * kTmaRows * 4 +
-           (size_t)max_slots * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
-}
-
-// Item range [beg, end) of CTA c out of G (see GemvTmaArgs::split).
-__host__ __device__ __forceinline__ void gemv_tma_range(int64_t nblocks, int slices, int split, int64_t c, int64_t G,
-                                                        int64_t &beg, int64_t &end) {
-    if (split) {
-        const int64_t items = nblocks * slices;
-        beg = items * c / G;
-        end = items * (c + 1) / G;
-    } else {
-        beg = nblocks * c / G * slices;
-        end = nblocks * (c + 1) / G * slices;
-    }
-}
-
-// The CTA whose range holds item i (split mode): the largest c with
-// floor(c * I / G) <= i.
-__device__ __forceinline__ int64_t gemv_tma_owner(int64_t i, int64_t items, int64_t G) {
-    const int64_t c = ((i + 1) * G - 1) / items;
-    return c < G - 1 ? c : G - 1;
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+           (size_t)tokens * slices * kTmaSliceK + (size_t)max_blocks_cta * tokens * kTmaRows * 4 +
+           (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -282,13 +248,11 @@ __device__ __forceinline__ void stage_qlin_bf16_tokens(int8_t *qlin, int *qslice
 
 // ------------------------------------------------------------------ kernel
 
-// Every variant but the 8-warp, 8-token one fits twice on an SM (at most 32K
-// registers and, by the plan, under half the shared memory): the next
-// launch's CTA is resident beside this one and has its weights in flight
-// before this launch completes.  (8 warps x 8 tokens needs more registers
-// than that without spilling.)
+// Resident CTAs the register budget leaves room for: two for the 8-warp and
+// smaller variants (up to 4 tokens), so that the next launch's CTAs can start
+// (and request their weights) on an SM while this launch is finishing there.
 template <int W, int MT>
-constexpr int gemv_tma_min_blocks() { return (W == 8 && MT == 8) ? 1 : 2; }
+constexpr int gemv_tma_min_blocks() { return (W <= 8 && MT <= 4) ? 2 : 1; }
 
 template <int XMODE, int W, int MT>
 __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
@@ -300,7 +264,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     // the descriptor fetch is the first long latency of the launch: start it now
     if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     const int ns = a.ns, slices = a.slices;
-    const int64_t cid = blockIdx.x, G = gridDim.x;
+    const int64_t cid = blockIdx.x, ncl = gridDim.x;  // row blocks cid, cid + ncl, ...
     const int64_t kq = (int64_t)slices * kTmaSliceK;
 
     // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8
@@ -309,33 +273,32 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kTmaBoxBytes);   // [MT][kq]
     int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][32]
-    int *done = accs + a.max_slots * MT * kTmaRows;                            // [slot] items done
-    int *qslice = done + a.max_slots;                                          // [MT][slices]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(qslice + MT * slices + ((a.max_slots + MT * slices) & 1));
+    int *done = accs + a.max_blocks_cta * MT * kTmaRows;                       // [slot] items done
+    int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
+    uint64_t *bars =
+        reinterpret_cast<uint64_t *>(qslice + MT * slices + ((a.max_blocks_cta + MT * slices) & 1));
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // this CTA's items [beg, end), in (row block, slice) order; slot = row block - b0
-    int64_t beg, end;
-    gemv_tma_range(a.nblocks, slices, a.split, cid, G, beg, end);
-    const int64_t items = end - beg;
-    const int64_t b0 = beg / slices;
-    const int nslots = items > 0 ? (int)((end - 1) / slices - b0 + 1) : 0;
-    // this warp's items: a contiguous part of the CTA's range
+    // this CTA's items, in (row block, slice) order
+    const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
+    const int64_t items = nb_cta * slices;
+    const int nslots = (int)nb_cta;
+    // this warp's items: a contiguous range of the CTA's items
     const int64_t ipw = ceil_div(items, W);
-    const int64_t it_begin = beg + min(items, warp * ipw);
-    const int n_items = (int)(min(end, it_begin + ipw) - it_begin);
+    const int64_t it_begin = min(items, warp * ipw);
+    const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
     uint64_t *mybar = bars + warp * ns;
     uint8_t *myring = ring + warp * ns * kTmaBoxBytes;
 
-    // cursor over the warp's items: (row block, slice)
-    int64_t iblk = it_begin / slices;
-    int ij = (int)(it_begin - iblk * slices);
+    // cursor over the warp's items: (slot, slice); row block = cid + slot * ncl
+    int islot = (int)(it_begin / slices), ij = (int)(it_begin - (int64_t)islot * slices);
     auto issue_next = [&](int s) {
+        const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * kTmaRows;
         mbar_arrive_expect_tx(&mybar[s], kTmaBoxBytes);
-        tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)(iblk * kTmaRows), &mybar[s]);
+        tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
         if (++ij == slices) {
             ij = 0;
-            ++iblk;
+            ++islot;
         }
     };
     // weights do not depend on the previous kernel: request them before waiting
@@ -348,7 +311,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
             if (s == 0 && warp == 0 && a.test_stall) {  // skip the request: nothing completes this stage
                 if (++ij == slices) {
                     ij = 0;
-                    ++iblk;
+                    ++islot;
                 }
                 continue;
             }
@@ -359,7 +322,6 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
     pdl_launch_dependents();
     pdl_wait();
-    if (items == 0) return;  // no work (more CTAs than row blocks); nothing requested
 
     float sc[MT];
     if (XMODE == 1 && MT > 1) stage_qlin_bf16_tokens<MT>(qlin, qslice, slices, red, a.x, a.M, a.K, kq, sc);
@@ -387,29 +349,14 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
         f[t] = 0.0f;
         if (t < a.M && a.y_bf16 != nullptr) f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
     }
-    auto store = [&](int64_t n, int t, int tot) {
-        if (t < a.M && n < a.N) {
-            if (a.y_bf16 != nullptr)
-                a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
-            else
-                a.y_i32[(int64_t)t * a.N + n] = tot;
-        }
-    };
 
     int acc[MT][4], corr[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
     int ncontrib = 0;
-    // folds this warp's partial sums of row block `blk` into shared memory;
-    // the warp completing the CTA's items of the block finishes it: stores the
-    // results of a block the CTA owns whole, publishes the CTA's partial sums
-    // of a block that began in an earlier CTA, and, in the CTA holding the
-    // block's first item, adds the later CTAs' published sums and stores
-    auto flush = [&](int64_t blk) {
-        const int sl = (int)(blk - b0);
-        const int64_t lo = blk * slices > beg ? blk * slices : beg;
-        const int64_t hi = (blk + 1) * slices < end ? (blk + 1) * slices : end;
-        const int cnt = (int)(hi - lo);
+    // folds this warp's partial sums of slot `sl` into shared memory; the warp
+    // completing the slot's items writes its results
+    auto flush = [&](int sl) {
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
             const int v = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) - corr[t];
@@ -418,58 +365,19 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
         __threadfence_block();
         __syncwarp();
         int fin = 0;
-        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == cnt);
+        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == slices);
         fin = __shfl_sync(0xffffffffu, fin, 0);
         if (fin) {
             __threadfence_block();
-            const int64_t n = blk * kTmaRows + lane;
-            int tot[MT];
+            const int64_t n = (a.blk_begin + cid + (int64_t)sl * ncl) * kTmaRows + lane;
 #pragma unroll
-            for (int t = 0; t < MT; ++t) tot[t] = atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], 0);
-            if (cnt == slices) {
-#pragma unroll
-                for (int t = 0; t < MT; ++t) store(n, t, tot[t]);
-            } else if (lo > blk * slices) {
-                // the block began in an earlier CTA: publish this CTA's share
-#pragma unroll
-                for (int t = 0; t < MT; ++t) a.rec[(cid * MT + t) * kTmaRows + lane] = tot[t];
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release_u32(a.flags + cid, a.epoch);
-            } else {
-                // the block's first item is here: add the shares of the CTAs
-                // that hold its later items (published when each finished its
-                // first row block), then store
-                const int64_t items_all = a.nblocks * slices;
-                const int64_t c_hi = gemv_tma_owner((blk + 1) * slices - 1, items_all, G);
-                bool ok = true;
-                for (int64_t c2 = cid + 1; c2 <= c_hi && ok; ++c2) {
-                    uint32_t fl = 0;
-                    if (lane == 0) {
-                        fl = ld_acquire_u32(a.flags + c2);
-                        if (fl != a.epoch) {
-                            const uint64_t t0 = global_timer_ns();
-                            while ((fl = ld_acquire_u32(a.flags + c2)) != a.epoch) {
-                                if (global_timer_ns() - t0 > kWaitLimitNs) break;
-                                __nanosleep(32);
-                            }
-                        }
-                    }
-                    fl = __shfl_sync(0xffffffffu, fl, 0);
-                    if (fl != a.epoch) {
-                        if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) tot[t] += __ldcg(a.rec + (c2 * MT + t) * kTmaRows + lane);
-                    __syncwarp();
-                    if (lane == 0) a.flags[c2] = 0u;  // consumed: a replay with the same tag starts clean
-                }
-                if (ok) {
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) store(n, t, tot[t]);
+            for (int t = 0; t < MT; ++t) {
+                const int tot = atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], 0);
+                if (t < a.M && n < a.N) {
+                    if (a.y_bf16 != nullptr)
+                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
+                    else
+                        a.y_i32[(int64_t)t * a.N + n] = tot;
                 }
             }
         }
@@ -479,8 +387,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     };
 
     // consume cursor
-    int64_t cblk = it_begin / slices;
-    int cj = (int)(it_begin - cblk * slices);
+    int cslot = (int)(it_begin / slices), cj = (int)(it_begin - (int64_t)cslot * slices);
     int s = 0;
     uint32_t phase = 0;
     for (int n = 0; n < n_items; ++n) {
@@ -538,9 +445,9 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
             phase ^= 1u;
         }
         if (++cj == slices || n + 1 == n_items) {
-            flush(cblk);
+            flush(cslot);
             cj = 0;
-            ++cblk;
+            ++cslot;
         }
     }
 }

@@ -102,18 +102,27 @@ __device__ __forceinline__ float quant_row(const uint16_t *__restrict__ xr, int6
     const bool qvec = (reinterpret_cast<uintptr_t>(qr) & 7) == 0;
     const int64_t nw = vec ? K / 8 : 0;  // whole 16-byte words of the row
 
+    // every load of the row is issued before the first is used: one memory
+    // round trip for the held words (and one per further batch), not one per word
     uint4 held[kQuantHeld];
-    float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < kQuantHeld; ++i) {
         const int64_t c = t + (int64_t)i * kTeam;
-        if (c < nw) {
-            held[i] = *reinterpret_cast<const uint4 *>(xr + 8 * c);
-            amax = amax8(held[i], amax);
-        }
+        held[i] = c < nw ? *reinterpret_cast<const uint4 *>(xr + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
     }
-    for (int64_t c = t + (int64_t)kQuantHeld * kTeam; c < nw; c += kTeam)
-        amax = amax8(*reinterpret_cast<const uint4 *>(xr + 8 * c), amax);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kQuantHeld; ++i) amax = amax8(held[i], amax);
+    for (int64_t c0 = t + (int64_t)kQuantHeld * kTeam; c0 < nw; c0 += (int64_t)4 * kTeam) {
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t c = c0 + (int64_t)i * kTeam;
+            v[i] = c < nw ? *reinterpret_cast<const uint4 *>(xr + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = amax8(v[i], amax);
+    }
     for (int64_t k = nw * 8 + t; k < K; k += kTeam) amax = fmaxf(amax, fabsf(bf16_bits_to_float(xr[k])));
     amax = team_max<WPT>(amax, fred, team, wt);
     const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
@@ -132,8 +141,19 @@ __device__ __forceinline__ float quant_row(const uint16_t *__restrict__ xr, int6
         const int64_t c = t + (int64_t)i * kTeam;
         if (c < nw) put8(c, quant8(held[i], sc, sum));
     }
-    for (int64_t c = t + (int64_t)kQuantHeld * kTeam; c < nw; c += kTeam)
-        put8(c, quant8(*reinterpret_cast<const uint4 *>(xr + 8 * c), sc, sum));
+    for (int64_t c0 = t + (int64_t)kQuantHeld * kTeam; c0 < nw; c0 += (int64_t)4 * kTeam) {
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t c = c0 + (int64_t)i * kTeam;
+            v[i] = c < nw ? *reinterpret_cast<const uint4 *>(xr + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t c = c0 + (int64_t)i * kTeam;
+            if (c < nw) put8(c, quant8(v[i], sc, sum));
+        }
+    }
     for (int64_t k = nw * 8 + t; k < K; k += kTeam) {
         const int8_t qi = quant_one(bf16_bits_to_float(xr[k]), sc);
         qr[k] = qi;

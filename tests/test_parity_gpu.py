@@ -190,7 +190,7 @@ def test_gemv_tma_largest_k_extremes():
     import sys
     from conftest import ROOT
     env = dict(os.environ)
-    env["BITNET_GEMV_TUNE"] = "0,0,0,0,-1,0,-1,1,0,4"  # TMA GEMV, 4 warps, ring of one box
+    env["BITNET_GEMV_TUNE"] = "0,0,0,0,-1,0,5,1"  # TMA GEMV variant of 4 warps, ring of one box
     r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + TMA_MAX_K_CHILD], env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]

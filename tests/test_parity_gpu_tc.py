@@ -129,3 +129,17 @@ def test_tc_every_tile_width(tile, S):
     res = json.loads(r.stdout.strip().splitlines()[-1])
     assert res.pop("device_error") == 0
     assert all(res.values()), res
+
+
+def test_bitlinear_with_quantisation_inside_the_gemm_launch():
+    """The alternative prefill path (tuning field fuse = 1): the GEMM launch
+    quantises the activations itself, its CTAs meeting at a grid barrier
+    before the first activation load; same cases, guard bands and checks."""
+    env = dict(os.environ)
+    env["BITNET_GEMV_TUNE"] = "0,0,0,0,-1,0,-1,0,1"
+    r = subprocess.run([sys.executable, "-c", "ROOT = " + repr(ROOT) + "\n" + CHILD], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert res.pop("device_error") == 0
+    assert all(res.values()), res

@@ -1,10 +1,10 @@
 """Parity of the TMA-staged decode GEMV under every launch variant.
 
 A child process forces the variant (BITNET_GEMV_TUNE, read once per process:
-warps per CTA, ring depth, whole row blocks per CTA or row blocks split across
-CTAs) on shapes with ragged row blocks (N not a multiple of 32), partial
-K-slices (K_pad/4 not a multiple of 128), a single row block, several row
-blocks per CTA, and 1, 3 or 8 tokens; int32 and BitLinear outputs.
+warps per CTA, ring depth, CTAs per SM) on shapes with ragged row blocks (N
+not a multiple of 32), partial K-slices (K_pad/4 not a multiple of 128), a
+single row block, several row blocks per CTA, and 1, 3 or 8 tokens; int32 and
+BitLinear outputs.
 """
 import json
 import os
@@ -53,17 +53,14 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,tma,ring,split,warps": for
-# the TMA GEMV, ring = boxes in flight per warp (0: planner), split = -1
-# planner / 0 whole row blocks per CTA / 1 an even split of all items (row
-# blocks spanning CTAs meet in the workspace), warps = 4, 8, 12 or 16 (4 and 8
-# only for 3 and 8 tokens; other values keep the planner's)
-@pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",                # the planner's own choice
-                                  "0,0,0,0,-1,0,-1,0,1,16",         # split, 16 warps
-                                  "0,0,0,0,-1,0,-1,1,1,4",          # split, 4 warps, ring of 1
-                                  "0,0,0,0,-1,0,-1,2,1,12",         # split, 12 warps, ring of 2
-                                  "0,0,0,0,-1,0,-1,4,0,8",          # whole blocks, 8 warps, ring of 4
-                                  "0,0,0,0,-1,0,-1,1,0,16"])        # whole blocks, 16 warps, ring of 1
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring": variant
+# 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp)
+@pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
+                                  "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
+                                  "0,0,0,0,-1,0,3",      # 16 warps, ring up to 2
+                                  "0,0,0,2,-1,0,4",      # 8 warps, ring up to 2, 2 CTAs per SM
+                                  "0,0,0,0,-1,0,5",      # 4 warps, ring up to 4
+                                  "0,0,0,0,-1,0,2,1"])   # 12 warps, ring of 1
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
