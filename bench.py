@@ -579,16 +579,15 @@ def run_ours(args, rank, world, dist):
                      "duration": "mean per-call time of each shape in a graph of back-to-back calls over rotating "
                                  "weight copies (CUDA events)"},
         "clocks": clk,
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps,
-                "note": "every step: the eight shapes' int8 activations copied in from pinned host memory (one "
-                        "copy), the eight public API calls, their int32 results copied out to pinned host memory "
-                        "(one copy), stream synchronised; packed weights resident",
-                "c_loop": {"value": round(e2e_c_value, 2), "unit": "GB/s",
-                           "us_per_step": round(e2e_c_ms * 1e3 / e2e_steps, 2),
-                           "note": "the same copies and C-ABI calls driven from C (bench_e2e.cu): library and "
-                                   "runtime overhead without the Python binding"},
-                "python_us_per_step": round(e2e_ms * 1e3 / e2e_steps, 2)},
+        "e2e": {"value": round(e2e_c_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "us_per_step": round(e2e_c_ms * 1e3 / e2e_steps, 2),
+                "note": "through the C ABI with host buffers (bench_e2e.cu): every step copies the eight shapes' "
+                        "int8 activations in from pinned host memory (one copy), makes the eight bitnet_w2a8_gemm "
+                        "calls, copies their int32 results out to pinned host memory (one copy) and synchronises "
+                        "the stream; packed weights resident",
+                "python": {"value": round(e2e_value, 2), "unit": "GB/s",
+                           "us_per_step": round(e2e_ms * 1e3 / e2e_steps, 2),
+                           "note": "the same step through the Python binding (torch tensors, ctypes)"}},
         "gpu_launches": int(launches_per_step * args.steps),
         "device_error": err,
         "details": details,

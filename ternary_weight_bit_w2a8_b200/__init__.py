@@ -82,9 +82,12 @@ def _ptr(t):
 
 def _stream(stream=None):
     import torch
-    if stream is None:
-        return torch.cuda.current_stream().cuda_stream
-    return stream.cuda_stream
+    if stream is not None:
+        return stream.cuda_stream
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)  # no Stream object per call
+    if raw is not None:
+        return raw(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _dev(t, name):

@@ -108,10 +108,12 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream
 // ------------------------------------------------------------------ activation quantisation
 // Teams of 1..8 warps per token: about a thousand warps in flight whatever M
 // (one warp per token from 1024 tokens up), so the pass is one wave that reads
-// each row from HBM once.
+// each row from HBM once, and wide enough teams that a thread holds all of
+// its words of the row (one load round trip).
 int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_t *q, int64_t ldq, bool zero_pad,
                  float *s, int32_t *rowsum, cudaStream_t st) {
-    const int wpt = M >= 1024 ? 1 : (M >= 512 ? 2 : (M >= 256 ? 4 : 8));
+    int wpt = M >= 1024 ? 1 : (M >= 512 ? 2 : (M >= 256 ? 4 : 8));
+    while (wpt < 8 && ceil_div(K, 8) > (int64_t)kQuantHeld * 32 * wpt) wpt *= 2;
     const int64_t teams_per_cta = kThreads / (32 * wpt);
     int64_t grid = ceil_div(M, teams_per_cta);
     const int64_t cap = (int64_t)dev->sm_count * (2048 / kThreads);

@@ -98,18 +98,9 @@ __device__ __forceinline__ void stage_q_int8(uint4 *qs, const int8_t *qrow, int6
 // Thread t owns the 16-value pieces t, t + blockDim, ...; up to kHeld of them
 // stay in registers between the absmax pass and the quantise pass.
 __device__ __forceinline__ void quant16(const uint4 &lo, const uint4 &hi, float sc, uint4 &out) {
-    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int8_t a = quant_one(__uint_as_float(w[2 * i] << 16), sc);
-        const int8_t b = quant_one(__uint_as_float(w[2 * i] & 0xffff0000u), sc);
-        const int8_t c = quant_one(__uint_as_float(w[2 * i + 1] << 16), sc);
-        const int8_t d = quant_one(__uint_as_float(w[2 * i + 1] & 0xffff0000u), sc);
-        o[i] = (uint32_t)(uint8_t)a | ((uint32_t)(uint8_t)b << 8) | ((uint32_t)(uint8_t)c << 16) |
-               ((uint32_t)(uint8_t)d << 24);
-    }
-    out = make_uint4(o[0], o[1], o[2], o[3]);
+    int unused = 0;
+    const uint2 a = quant8<false>(lo, sc, unused), b = quant8<false>(hi, sc, unused);
+    out = make_uint4(a.x, a.y, b.x, b.y);
 }
 
 __device__ __forceinline__ float amax16(const uint4 &lo, const uint4 &hi, float m) {

@@ -13,12 +13,24 @@ namespace bitnet {
 
 constexpr float kQuantEps = 1e-5f;
 
-__device__ __forceinline__ int8_t quant_one(float x, float sc) {
-    float r = rintf(__fmul_rn(x, sc));
-    if (r != r) r = 0.0f;
-    r = r > 127.0f ? 127.0f : r;
-    r = r < -128.0f ? -128.0f : r;
-    return (int8_t)r;
+// clamp(rne(x * sc), -128, 127), NaN to 0: one fp32 multiply and one
+// conversion (cvt.rni.s8.f32 rounds to nearest even, saturates to the int8
+// range and turns NaN into 0), returned sign-extended in an int.
+__device__ __forceinline__ int quant_i(float x, float sc) {
+    int r;
+    asm("cvt.rni.s8.f32 %0, %1;" : "=r"(r) : "f"(__fmul_rn(x, sc)));
+    return r;
+}
+
+__device__ __forceinline__ int8_t quant_one(float x, float sc) { return (int8_t)quant_i(x, sc); }
+
+// Low bytes of four ints in one word, a in byte 0.
+__device__ __forceinline__ uint32_t pack4_b0(int a, int b, int c, int d) {
+    uint32_t ab, cd, r;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(ab) : "r"(a), "r"(b));
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(cd) : "r"(c), "r"(d));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(ab), "r"(cd));
+    return r;
 }
 
 // |x| maximum over the 8 bf16 values of a 16-byte word.
@@ -32,19 +44,22 @@ __device__ __forceinline__ float amax8(const uint4 &v, float m) {
     return m;
 }
 
-// The 8 codes of a 16-byte word of bf16 values (low byte = lowest k), and
-// their sum added to `sum`.
+// The 8 codes of a 16-byte word of bf16 values (low byte = lowest k), and,
+// when SUM, their sum added to `sum`.
+template <bool SUM = true>
 __device__ __forceinline__ uint2 quant8(const uint4 &v, float sc, int &sum) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[2] = {0u, 0u};
+    int c[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int8_t lo = quant_one(__uint_as_float(w[i] << 16), sc);
-        const int8_t hi = quant_one(__uint_as_float(w[i] & 0xffff0000u), sc);
-        sum += lo + hi;
-        o[i >> 1] |= ((uint32_t)(uint8_t)lo | ((uint32_t)(uint8_t)hi << 8)) << (16 * (i & 1));
+        c[2 * i] = quant_i(__uint_as_float(w[i] << 16), sc);
+        c[2 * i + 1] = quant_i(__uint_as_float(w[i] & 0xffff0000u), sc);
     }
-    return make_uint2(o[0], o[1]);
+    if (SUM) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum += c[i];
+    }
+    return make_uint2(pack4_b0(c[0], c[1], c[2], c[3]), pack4_b0(c[4], c[5], c[6], c[7]));
 }
 
 // A team of WPT warps quantises one token row at a time (a CTA of kThreads
@@ -139,7 +154,7 @@ __device__ __forceinline__ float quant_row(const uint16_t *__restrict__ xr, int6
 #pragma unroll
     for (int i = 0; i < kQuantHeld; ++i) {
         const int64_t c = t + (int64_t)i * kTeam;
-        if (c < nw) put8(c, quant8(held[i], sc, sum));
+        if (c < nw) put8(c, want_sum ? quant8<true>(held[i], sc, sum) : quant8<false>(held[i], sc, sum));
     }
     for (int64_t c0 = t + (int64_t)kQuantHeld * kTeam; c0 < nw; c0 += (int64_t)4 * kTeam) {
         uint4 v[4];
@@ -151,7 +166,7 @@ __device__ __forceinline__ float quant_row(const uint16_t *__restrict__ xr, int6
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int64_t c = c0 + (int64_t)i * kTeam;
-            if (c < nw) put8(c, quant8(v[i], sc, sum));
+            if (c < nw) put8(c, want_sum ? quant8<true>(v[i], sc, sum) : quant8<false>(v[i], sc, sum));
         }
     }
     for (int64_t k = nw * 8 + t; k < K; k += kTeam) {
