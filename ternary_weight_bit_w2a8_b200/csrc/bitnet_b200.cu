@@ -37,7 +37,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[22] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    size_t tma_max_dyn[40] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[2 * 10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -105,30 +105,6 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// ------------------------------------------------------------------ activation quantisation
-// Teams of 1..8 warps per token: about a thousand warps in flight whatever M
-// (one warp per token from 1024 tokens up), so the pass is one wave that reads
-// each row from HBM once, and wide enough teams that a thread holds all of
-// its words of the row (one load round trip).
-int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_t *q, int64_t ldq, bool zero_pad,
-                 float *s, int32_t *rowsum, cudaStream_t st) {
-    int wpt = M >= 1024 ? 1 : (M >= 512 ? 2 : (M >= 256 ? 4 : 8));
-    while (wpt < 8 && ceil_div(K, 8) > (int64_t)kQuantHeld * 32 * wpt) wpt *= 2;
-    const int64_t teams_per_cta = kThreads / (32 * wpt);
-    int64_t grid = ceil_div(M, teams_per_cta);
-    const int64_t cap = (int64_t)dev->sm_count * (2048 / kThreads);
-    if (grid > cap) grid = cap;
-    const dim3 g((unsigned)grid), b(kThreads);
-    cudaError_t e;
-    switch (wpt) {
-        case 1: e = launch_pdl(quant_act_kernel<1>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
-        case 2: e = launch_pdl(quant_act_kernel<2>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
-        case 4: e = launch_pdl(quant_act_kernel<4>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
-        default: e = launch_pdl(quant_act_kernel<8>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
-    }
-    return launched(e);
-}
-
 // ------------------------------------------------------------------ fill (K == 0)
 template <typename T>
 __global__ void __launch_bounds__(kThreads) fill_kernel(T *p, int64_t n, T v) {
@@ -143,13 +119,15 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
-// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse"
+// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores"
 // (register GEMV: G, R, U, ctas, prefetch, S; TMA GEMV: tma = 0 off or
-// 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth; tensor-core GEMM:
-// R < 0 variant, S K-splits, fuse = 1 quantises BitLinear activations inside
-// the GEMM launch)
+// 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth, rows per block 16 or
+// 32, cores = 1 the co-residency mode (see tma_plan); tensor-core GEMM: R < 0
+// variant, S K-splits, fuse = 1 quantises BitLinear activations inside the
+// GEMM launch; activation quantisation: qwpt warps per token, 1..8)
 struct GemvTune {
-    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1;
+    int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1, qwpt = 0, rows = 0,
+        cores = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -158,10 +136,36 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma, &t.ns,
-                   &t.fuse);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma,
+                   &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores);
     });
     return t;
+}
+
+// ------------------------------------------------------------------ activation quantisation
+// Teams of 1..8 warps per token: about a thousand warps in flight whatever M
+// (one warp per token from 1024 tokens up), so the pass is one wave that reads
+// each row from HBM once, and wide enough teams that a thread holds all of
+// its words of the row (one load round trip).
+int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_t *q, int64_t ldq, bool zero_pad,
+                 float *s, int32_t *rowsum, cudaStream_t st) {
+    int wpt = M >= 1024 ? 1 : (M >= 512 ? 2 : (M >= 256 ? 4 : 8));
+    while (wpt < 8 && ceil_div(K, 8) > (int64_t)kQuantHeld * 32 * wpt) wpt *= 2;
+    const int tw = gemv_tune().qwpt;
+    if (tw == 1 || tw == 2 || tw == 4 || tw == 8) wpt = tw;
+    const int64_t teams_per_cta = kThreads / (32 * wpt);
+    int64_t grid = ceil_div(M, teams_per_cta);
+    const int64_t cap = (int64_t)dev->sm_count * (2048 / kThreads);
+    if (grid > cap) grid = cap;
+    const dim3 g((unsigned)grid), b(kThreads);
+    cudaError_t e;
+    switch (wpt) {
+        case 1: e = launch_pdl(quant_act_kernel<1>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        case 2: e = launch_pdl(quant_act_kernel<2>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        case 4: e = launch_pdl(quant_act_kernel<4>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+        default: e = launch_pdl(quant_act_kernel<8>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
+    }
+    return launched(e);
 }
 
 inline int lanes_per_row(int nch) { return nch >= 128 ? 32 : (nch >= 48 ? 16 : 8); }
@@ -303,41 +307,46 @@ using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 // 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
 constexpr int kFusedQuantMaxTokens = 4;
 
-// Kernel of (mode, warps, tokens per launch): one token on 4, 8, 12 or 16
-// warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8 activations
-// (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16 activations
-// quantised in the kernel (xmode 1).  Slot in the shared-memory opt-in table:
-// MT == 1 ? xmode * 10 + W / 4 - 1 : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16);
-// -1 if none.
-int tma_kernel_slot(int xmode, int cfg, int mt) {
+// Kernel of (mode, warps, tokens per launch, rows per block): one token on 4,
+// 8, 12 or 16 warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8
+// activations (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16
+// activations quantised in the kernel (xmode 1); row blocks of 32 or 16 rows.
+// Slot in the kernel and shared-memory opt-in tables (-1 if none):
+// (rows == 16) * 20 + (MT == 1 ? xmode * 10 + W / 4 - 1
+//                              : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16)).
+int tma_kernel_slot(int xmode, int cfg, int mt, int rows) {
     const int W = kTmaCfg[cfg][0];
-    if (mt == 1) return xmode * 10 + W / 4 - 1;
+    const int base = rows == 16 ? 20 : 0;
+    if (mt == 1) return base + xmode * 10 + W / 4 - 1;
     if (W != 8 && W != 16) return -1;
     if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
-    return xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
+    return base + xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
 }
 
-TmaKernel tma_kernel_for(int xmode, int cfg, int mt) {
-    static const TmaKernel table[20] = {
-        gemv_tma_kernel<0, 4, 1>, gemv_tma_kernel<0, 8, 1>, gemv_tma_kernel<0, 12, 1>, gemv_tma_kernel<0, 16, 1>,
-        gemv_tma_kernel<0, 8, 2>, gemv_tma_kernel<0, 16, 2>, gemv_tma_kernel<0, 8, 4>, gemv_tma_kernel<0, 16, 4>,
-        gemv_tma_kernel<0, 8, 8>, gemv_tma_kernel<0, 16, 8>,
-        gemv_tma_kernel<1, 4, 1>, gemv_tma_kernel<1, 8, 1>, gemv_tma_kernel<1, 12, 1>, gemv_tma_kernel<1, 16, 1>,
-        gemv_tma_kernel<1, 8, 2>, gemv_tma_kernel<1, 16, 2>, gemv_tma_kernel<1, 8, 4>, gemv_tma_kernel<1, 16, 4>,
-        nullptr, nullptr};  // (bf16, 8 tokens): quantised beforehand instead
-    const int slot = tma_kernel_slot(xmode, cfg, mt);
+#define BITNET_TMA_VARIANTS(R)                                                                                   \
+    gemv_tma_kernel<0, 4, 1, R>, gemv_tma_kernel<0, 8, 1, R>, gemv_tma_kernel<0, 12, 1, R>,                     \
+        gemv_tma_kernel<0, 16, 1, R>, gemv_tma_kernel<0, 8, 2, R>, gemv_tma_kernel<0, 16, 2, R>,                \
+        gemv_tma_kernel<0, 8, 4, R>, gemv_tma_kernel<0, 16, 4, R>, gemv_tma_kernel<0, 8, 8, R>,                 \
+        gemv_tma_kernel<0, 16, 8, R>, gemv_tma_kernel<1, 4, 1, R>, gemv_tma_kernel<1, 8, 1, R>,                 \
+        gemv_tma_kernel<1, 12, 1, R>, gemv_tma_kernel<1, 16, 1, R>, gemv_tma_kernel<1, 8, 2, R>,                \
+        gemv_tma_kernel<1, 16, 2, R>, gemv_tma_kernel<1, 8, 4, R>, gemv_tma_kernel<1, 16, 4, R>,                \
+        nullptr, nullptr /* (bf16, 8 tokens): quantised beforehand instead */
+TmaKernel tma_kernel_for(int xmode, int cfg, int mt, int rows) {
+    static const TmaKernel table[40] = {BITNET_TMA_VARIANTS(32), BITNET_TMA_VARIANTS(16)};
+    const int slot = tma_kernel_slot(xmode, cfg, mt, rows);
     return slot < 0 ? nullptr : table[slot];
 }
+#undef BITNET_TMA_VARIANTS
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int rows) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    const int si = tma_kernel_slot(xmode, cfg, mt);
+    const int si = tma_kernel_slot(xmode, cfg, mt, rows);
     if (si < 0) return 0;
     size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, cfg, mt);
+        TmaKernel kern = tma_kernel_for(xmode, cfg, mt, rows);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -348,55 +357,76 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt) {
 }
 
 // Plan of the TMA GEMV, from the shape and B200 reference figures only (148
-// SMs, 227 KB of shared memory per CTA), so that what a shape needs does not
+// SMs, 228 KB of shared memory per SM), so that what a shape needs does not
 // depend on the device that runs it.
+//   - Row blocks of 32 rows; CTA c takes row blocks c, c + grid, ..., with at
+//     most 148 CTAs.
+//   - Variant (measured on B200): 16 warps x up to 2 boxes in flight, 12 x 3
+//     for rows of >= 32 K-slices; 8 or 16 warps for several tokens.  The ring
+//     is no deeper than the warp's items need.
+//   - One CTA per SM per launch, for every launch: its shared memory is padded
+//     past half an SM.  Programmatic dependent launch could otherwise start
+//     the next call's CTAs beside this call's, to request their weights early;
+//     that pays for a shape repeated alone when every SM holds one CTA of each
+//     launch (4736 x 2560: 2.44 -> 1.99 us per call; with 16-row blocks so
+//     that small shapes reach 148 CTAs too, 2560 x 2560: 2.13 -> 2.01 us), but
+//     in the benchmark's sequence of eight different shapes the calls then
+//     slow each other down (25.4 -> 30.5 us per step).  The tuning field
+//     `cores` = 1 selects that mode (16-row blocks where 32-row ones leave SMs
+//     idle, shallower rings for short calls so that two CTAs fit an SM).
 struct TmaPlan {
     bool use;
     int cfg, slices, max_blocks, grid;
     int ns;            // ring depth per warp
     int mt;            // tokens per launch (1, 2, 4, 8)
+    int rows;          // rows per block (32 or 16)
+    int64_t nblocks;
     size_t smem;
     int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
 };
 
 TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     constexpr int kRefSMs = 148;
-    constexpr size_t kRefSmemOptin = 232448;
+    constexpr size_t kRefSmemOptin = 232448;  // one CTA per SM
+    constexpr size_t kRefSmemHalf = 113664;   // two CTAs per SM (1 KB reserved and 1 KB static memory each)
+    const GemvTune &tn = gemv_tune();
     TmaPlan p{};
-    const int tune = gemv_tune().tma;
+    const int tune = tn.tma;
     if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
     // a lane accumulates one row's whole K: |acc_j| <= 4096 * K_pad stays
     // inside int32 for K_pad <= 2^19 (shared memory caps K lower still)
     if (k_pad(K) > ((int64_t)1 << 19)) return p;
     p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
     const int64_t row_bytes = packed_row_bytes(K);
-    const int64_t nblocks = ceil_div(N, kTmaRows);
+    // co-residency mode (tuning field `cores` = 1, see above); eight tokens
+    // keep 32-row blocks: their 16-warp variant has no registers to spare for
+    // the second lane of a row
+    const bool cores = tn.cores == 1;
+    p.rows = (!cores || ceil_div(N, kTmaRows) >= kRefSMs || p.mt == 8) ? 32 : 16;
+    if (tn.rows == 16 || tn.rows == 32) p.rows = tn.rows;
+    p.nblocks = ceil_div(N, p.rows);
     p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
-    // variant (measured on B200 over sequences of different shapes, as in a
-    // decode step): 16 x 2, and 12 x 3 for rows of K >= 16384.  Variants that
-    // let two CTAs share an SM win on a shape repeated alone but lose in a
-    // mixed sequence, where the scheduler can then stack two CTAs of one
-    // launch on an SM.
     if (tune >= 1 && tune <= kTmaNumCfg)
         p.cfg = tune - 1;
     else
         p.cfg = p.slices >= 32 ? 1 : 2;
     if (p.mt > 1 && kTmaCfg[p.cfg][0] != 8 && kTmaCfg[p.cfg][0] != 16) p.cfg = 2;  // several tokens: 8 or 16 warps
     const int W = kTmaCfg[p.cfg][0], NS = kTmaCfg[p.cfg][1];
-    // at most one CTA per SM per launch (BITNET_GEMV_TUNE's ctas field
-    // overrides): each SM keeps room for a CTA of the next launch, which then
-    // starts and requests its weights while this one finishes
-    const int per_sm = gemv_tune().ctas > 0 ? gemv_tune().ctas : 1;
+    // BITNET_GEMV_TUNE's ctas field: CTAs per SM per launch (1 by default)
+    const int per_sm = tn.ctas > 0 ? tn.ctas : 1;
     const int64_t gmax = (int64_t)kRefSMs * per_sm;
-    p.grid = (int)(nblocks < gmax ? nblocks : gmax);
-    p.max_blocks = (int)ceil_div(nblocks, p.grid);
-    // ring depth: no more boxes per warp than its items (a small launch then
-    // needs little shared memory and leaves room beside it)
+    p.grid = (int)(p.nblocks < gmax ? p.nblocks : gmax);
+    p.max_blocks = (int)ceil_div(p.nblocks, p.grid);
     const int64_t ipw = ceil_div((int64_t)p.max_blocks * p.slices, W);
     p.ns = (int)(ipw < NS ? (ipw < 1 ? 1 : ipw) : NS);
-    if (gemv_tune().ns > 0) p.ns = gemv_tune().ns < NS ? gemv_tune().ns : NS;
-    p.smem = gemv_tma_smem_bytes(W, p.ns, p.slices, p.max_blocks, p.mt);
+    if (tn.ns > 0) p.ns = tn.ns < NS ? tn.ns : NS;
+    auto bytes = [&](int ns) { return gemv_tma_smem_bytes(W, ns, p.slices, p.max_blocks, p.mt, p.rows); };
+    if (cores && p.grid >= kRefSMs && ipw <= 4)
+        while (p.ns > 1 && bytes(p.ns) > kRefSmemHalf) --p.ns;
+    p.smem = bytes(p.ns);
     if (p.smem > kRefSmemOptin - 1024) return TmaPlan{};
+    // one CTA per SM: always, or (co-residency mode) when the launch leaves SMs idle
+    if ((!cores || p.grid < kRefSMs) && p.smem <= kRefSmemHalf) p.smem = kRefSmemHalf + 4096;
     p.use = true;
     return p;
 }
@@ -404,14 +434,14 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
                     const TmaPlan &tp, cudaStream_t st) {
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt);
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt, tp.rows);
     if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
-    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt))
+    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt, tp.rows))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
     if (!encode_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes,
-                   kTmaSliceBytes, kTmaRows, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+                   kTmaSliceBytes, (uint32_t)tp.rows, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
         return BITNET_ERR_CUDA;
     // test hook (BITNET_TEST_STALL=1): the first TMA launch of the process
     // makes one wait run out, exercising the device-timeout path
@@ -431,7 +461,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.K = K;
     a.slices = tp.slices;
     a.blk_begin = 0;
-    a.nblocks = ceil_div(N, kTmaRows);
+    a.nblocks = tp.nblocks;
     a.max_blocks_cta = tp.max_blocks;
     a.ns = tp.ns;
     a.y_i32 = y_i32;

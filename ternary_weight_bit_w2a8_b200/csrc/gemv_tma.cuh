@@ -5,9 +5,12 @@
 // on codes scaled by 4^j, activation-sum correction); what differs is how the
 // weights reach the lanes:
 //   - The packed matrix is a 2-D byte tensor [N rows, K_pad/4 bytes].  A TMA
-//     box is 32 rows x 128 bytes (512 k) = 4 KB, written to shared memory with
-//     the 128-byte swizzle, so lane r reading 16-byte chunk c of its own row r
-//     (address r*128 + ((c ^ (r & 7)) * 16)) is free of bank conflicts.
+//     box is ROWS rows x 128 bytes (512 k): 32 rows (4 KB, one lane per row)
+//     or 16 rows (2 KB, two lanes per row, each taking half of the row's 8
+//     chunks), written to shared memory with the 128-byte swizzle, so a lane
+//     reading 16-byte chunk c of box row r (address r*128 + ((c ^ (r & 7)) *
+//     16)) is free of bank conflicts.  16-row blocks give shapes of fewer than
+//     148 32-row blocks one block for every SM.
 //   - Work items are (32-row block, 128-byte K-slice) pairs.  CTA b owns row
 //     blocks b, b + gridDim.x, ...; its items, in (row block, slice) order, are
 //     split into equal contiguous ranges, one per warp, which keeps every warp
@@ -39,10 +42,9 @@
 
 namespace bitnet {
 
-constexpr int kTmaRows = 32;                                // rows per box (one per lane)
+constexpr int kTmaRows = 32;                                // rows per box at one lane per row
 constexpr int kTmaSliceBytes = 128;                         // packed bytes per row per box
 constexpr int kTmaSliceK = kTmaSliceBytes * 4;              // k values per box
-constexpr int kTmaBoxBytes = kTmaRows * kTmaSliceBytes;     // 4 KB
 constexpr uint64_t kWaitLimitNs = 1000000000ull;            // 1 s per wait
 
 struct GemvTmaArgs {
@@ -62,12 +64,13 @@ struct GemvTmaArgs {
     int test_stall;       // test hook: warp 0 never requests its first box, so its first wait times out
 };
 
-// Dynamic shared memory of a launch: ring of warps x stages boxes, linear
-// activations, per-row-block accumulators and counters, slice sums, mbarriers.
+// Dynamic shared memory of a launch: ring of warps x stages boxes of `rows`
+// rows, linear activations, per-row-block accumulators and counters, slice
+// sums, mbarriers.
 __host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta,
-                                                      int tokens = 1) {
-    return 1024 /* alignment slack */ + (size_t)warps * stages * kTmaBoxBytes +
-           (size_t)tokens * slices * kTmaSliceK + (size_t)max_blocks_cta * tokens * kTmaRows * 4 +
+                                                      int tokens = 1, int rows = kTmaRows) {
+    return 1024 /* alignment slack */ + (size_t)warps * stages * rows * kTmaSliceBytes +
+           (size_t)tokens * slices * kTmaSliceK + (size_t)max_blocks_cta * tokens * rows * 4 +
            (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
 }
 
@@ -248,16 +251,21 @@ __device__ __forceinline__ void stage_qlin_bf16_tokens(int8_t *qlin, int *qslice
 
 // ------------------------------------------------------------------ kernel
 
-// Resident CTAs the register budget leaves room for: two for the 8-warp and
-// smaller variants (up to 4 tokens), so that the next launch's CTAs can start
-// (and request their weights) on an SM while this launch is finishing there.
+// Resident CTAs the register budget leaves room for: two for every variant of
+// up to two tokens and for the 8-warp ones of up to four, so that the next
+// launch's CTA can start beside this one's on an SM (and request its weights)
+// while this launch finishes there.
 template <int W, int MT>
-constexpr int gemv_tma_min_blocks() { return (W <= 8 && MT <= 4) ? 2 : 1; }
+constexpr int gemv_tma_min_blocks() { return (MT <= 2 || (W <= 8 && MT <= 4)) ? 2 : 1; }
 
-template <int XMODE, int W, int MT>
+template <int XMODE, int W, int MT, int ROWS>
 __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
     static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8, "tokens per launch");
+    static_assert(ROWS == 32 || ROWS == 16, "rows per box");
+    constexpr int kLPR = kTmaRows / ROWS;               // lanes per row
+    constexpr int kCPL = 8 / kLPR;                      // 16-byte chunks per lane per box
+    constexpr int kBoxBytes = ROWS * kTmaSliceBytes;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ float red[(XMODE == 1 ? MT : 1) * 32];
@@ -271,14 +279,15 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     // rows of 128 bytes), computed on the shared-window address so that every
     // pointer below stays a shared-memory pointer
     uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kTmaBoxBytes);   // [MT][kq]
-    int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][32]
-    int *done = accs + a.max_blocks_cta * MT * kTmaRows;                       // [slot] items done
+    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kBoxBytes);      // [MT][kq]
+    int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][ROWS]
+    int *done = accs + a.max_blocks_cta * MT * ROWS;                           // [slot] items done
     int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
     uint64_t *bars =
         reinterpret_cast<uint64_t *>(qslice + MT * slices + ((a.max_blocks_cta + MT * slices) & 1));
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int brow = lane / kLPR, part = lane % kLPR;  // this lane's box row and chunk half
     // this CTA's items, in (row block, slice) order
     const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
     const int64_t items = nb_cta * slices;
@@ -288,14 +297,14 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     const int64_t it_begin = min(items, warp * ipw);
     const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
     uint64_t *mybar = bars + warp * ns;
-    uint8_t *myring = ring + warp * ns * kTmaBoxBytes;
+    uint8_t *myring = ring + warp * ns * kBoxBytes;
 
     // cursor over the warp's items: (slot, slice); row block = cid + slot * ncl
     int islot = (int)(it_begin / slices), ij = (int)(it_begin - (int64_t)islot * slices);
     auto issue_next = [&](int s) {
-        const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * kTmaRows;
-        mbar_arrive_expect_tx(&mybar[s], kTmaBoxBytes);
-        tma_load_box(myring + s * kTmaBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
+        const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * ROWS;
+        mbar_arrive_expect_tx(&mybar[s], kBoxBytes);
+        tma_load_box(myring + s * kBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
         if (++ij == slices) {
             ij = 0;
             ++islot;
@@ -318,7 +327,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
             issue_next(s);
         }
     }
-    for (int i = threadIdx.x; i < nslots * MT * kTmaRows; i += blockDim.x) accs[i] = 0;
+    for (int i = threadIdx.x; i < nslots * MT * ROWS; i += blockDim.x) accs[i] = 0;
     for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
     pdl_launch_dependents();
     pdl_wait();
@@ -354,13 +363,15 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
 #pragma unroll
     for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
     int ncontrib = 0;
-    // folds this warp's partial sums of slot `sl` into shared memory; the warp
-    // completing the slot's items writes its results
+    // folds this warp's partial sums of slot `sl` into shared memory (the
+    // lanes sharing a row each add their half; the activation-sum correction
+    // is taken once per row); the warp completing the slot's items writes its
+    // results
     auto flush = [&](int sl) {
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
-            const int v = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) - corr[t];
-            atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], v);
+            const int v = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) - (part == 0 ? corr[t] : 0);
+            atomicAdd(&accs[(sl * MT + t) * ROWS + brow], v);
         }
         __threadfence_block();
         __syncwarp();
@@ -369,11 +380,11 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
         fin = __shfl_sync(0xffffffffu, fin, 0);
         if (fin) {
             __threadfence_block();
-            const int64_t n = (a.blk_begin + cid + (int64_t)sl * ncl) * kTmaRows + lane;
+            const int64_t n = (a.blk_begin + cid + (int64_t)sl * ncl) * ROWS + brow;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-                const int tot = atomicAdd(&accs[(sl * MT + t) * kTmaRows + lane], 0);
-                if (t < a.M && n < a.N) {
+                const int tot = atomicAdd(&accs[(sl * MT + t) * ROWS + brow], 0);
+                if (part == 0 && t < a.M && n < a.N) {
                     if (a.y_bf16 != nullptr)
                         a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
                     else
@@ -398,11 +409,12 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
                 mbar_wait_bounded(&mybar[(n + d) % ns], (uint32_t)((n + d) / ns) & 1u);
             break;
         }
-        const uint8_t *row = myring + s * kTmaBoxBytes + lane * kTmaSliceBytes;
+        const uint8_t *row = myring + s * kBoxBytes + brow * kTmaSliceBytes;
         const int8_t *qk = qlin + cj * kTmaSliceK;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (lane & 7)) << 4));
+        for (int cc = 0; cc < kCPL; ++cc) {
+            const int c = part * kCPL + cc;
+            const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (brow & 7)) << 4));
             if (MT == 1) {
                 const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
                 const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];

@@ -13,19 +13,29 @@ namespace bitnet {
 
 constexpr float kQuantEps = 1e-5f;
 
-// clamp(rne(x * sc), -128, 127), NaN to 0: one fp32 multiply and one
-// conversion (cvt.rni.s8.f32 rounds to nearest even, saturates to the int8
-// range and turns NaN into 0), returned sign-extended in an int.
-__device__ __forceinline__ int quant_i(float x, float sc) {
-    int r;
-    asm("cvt.rni.s8.f32 %0, %1;" : "=r"(r) : "f"(__fmul_rn(x, sc)));
-    return r;
+// clamp(rne(x * sc), -128, 127), NaN to 0, in full-rate fp32 arithmetic
+// (conversion instructions run at a fraction of that rate).  With sc =
+// 127 / max|x| the product lies in [-127, 127] up to one rounding, so no
+// clamp is needed: adding 1.5 * 2^23 rounds it to the nearest integer, ties
+// to even (the float spacing there is 1 and 1.5 * 2^23 is even), and leaves
+// that integer in the low mantissa bits.  Returns the word whose low byte
+// is the code (the bits of 1.5 * 2^23 for NaN, low byte 0); quant_val gives
+// the signed value.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+__device__ __forceinline__ uint32_t quant_bits(float x, float sc) {
+    const float v = __fmul_rn(x, sc);
+    const uint32_t b = __float_as_uint(__fadd_rn(v, kRoundMagic));
+    return v == v ? b : kRoundMagicBits;
 }
 
-__device__ __forceinline__ int8_t quant_one(float x, float sc) { return (int8_t)quant_i(x, sc); }
+__device__ __forceinline__ int quant_val(uint32_t bits) { return (int)(bits - kRoundMagicBits); }
 
-// Low bytes of four ints in one word, a in byte 0.
-__device__ __forceinline__ uint32_t pack4_b0(int a, int b, int c, int d) {
+__device__ __forceinline__ int8_t quant_one(float x, float sc) { return (int8_t)quant_val(quant_bits(x, sc)); }
+
+// Low bytes of four words in one word, a in byte 0.
+__device__ __forceinline__ uint32_t pack4_b0(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     uint32_t ab, cd, r;
     asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(ab) : "r"(a), "r"(b));
     asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(cd) : "r"(c), "r"(d));
@@ -49,15 +59,15 @@ __device__ __forceinline__ float amax8(const uint4 &v, float m) {
 template <bool SUM = true>
 __device__ __forceinline__ uint2 quant8(const uint4 &v, float sc, int &sum) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    int c[8];
+    uint32_t c[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        c[2 * i] = quant_i(__uint_as_float(w[i] << 16), sc);
-        c[2 * i + 1] = quant_i(__uint_as_float(w[i] & 0xffff0000u), sc);
+        c[2 * i] = quant_bits(__uint_as_float(w[i] << 16), sc);
+        c[2 * i + 1] = quant_bits(__uint_as_float(w[i] & 0xffff0000u), sc);
     }
     if (SUM) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sum += c[i];
+        for (int i = 0; i < 8; ++i) sum += quant_val(c[i]);
     }
     return make_uint2(pack4_b0(c[0], c[1], c[2], c[3]), pack4_b0(c[4], c[5], c[6], c[7]));
 }

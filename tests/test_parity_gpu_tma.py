@@ -53,14 +53,19 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring": variant
-# 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp)
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores":
+# variant 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp), rows
+# per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM)
 @pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
                                   "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
                                   "0,0,0,0,-1,0,3",      # 16 warps, ring up to 2
                                   "0,0,0,2,-1,0,4",      # 8 warps, ring up to 2, 2 CTAs per SM
                                   "0,0,0,0,-1,0,5",      # 4 warps, ring up to 4
-                                  "0,0,0,0,-1,0,2,1"])   # 12 warps, ring of 1
+                                  "0,0,0,0,-1,0,2,1",    # 12 warps, ring of 1
+                                  "0,0,0,0,-1,0,-1,0,-1,0,16",   # 16-row blocks (two lanes per row)
+                                  "0,0,0,0,-1,0,1,0,-1,0,16",    # 16-row blocks, 8 warps, ring up to 4
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,1",  # co-residency mode (16-row blocks below 148)
+                                  "0,0,0,0,-1,0,-1,0,-1,0,32,1"])  # co-residency mode, 32-row blocks
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
