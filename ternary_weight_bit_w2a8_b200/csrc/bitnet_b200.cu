@@ -37,7 +37,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[40] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    size_t tma_max_dyn[200] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[2 * 10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -119,15 +119,16 @@ struct GemvSplit {
     int64_t ws_bytes;
 };
 
-// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores"
+// optional override: BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores,mma"
 // (register GEMV: G, R, U, ctas, prefetch, S; TMA GEMV: tma = 0 off or
 // 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth, rows per block 16 or
-// 32, cores = 1 the co-residency mode (see tma_plan); tensor-core GEMM: R < 0
+// 32, cores = 1 the co-residency mode (see tma_plan), mma = 1 / 0 the MMA or
+// dp4a product for one token; tensor-core GEMM: R < 0
 // variant, S K-splits, fuse = 1 quantises BitLinear activations inside the
 // GEMM launch; activation quantisation: qwpt warps per token, 1..8)
 struct GemvTune {
     int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1, qwpt = 0, rows = 0,
-        cores = -1;
+        cores = -1, mma = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -136,8 +137,8 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S, &t.tma,
-                   &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S,
+                   &t.tma, &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores, &t.mma);
     });
     return t;
 }
@@ -307,46 +308,74 @@ using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 // 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
 constexpr int kFusedQuantMaxTokens = 4;
 
-// Kernel of (mode, warps, tokens per launch, rows per block): one token on 4,
-// 8, 12 or 16 warps, several tokens (MT = 2, 4, 8) on 8 or 16 warps, for int8
-// activations (xmode 0) and, up to kFusedQuantMaxTokens tokens, bf16
-// activations quantised in the kernel (xmode 1); row blocks of 32 or 16 rows.
-// Slot in the kernel and shared-memory opt-in tables (-1 if none):
-// (rows == 16) * 20 + (MT == 1 ? xmode * 10 + W / 4 - 1
-//                              : xmode * 10 + 4 + 2 * log2(MT / 2) + (W == 16)).
-int tma_kernel_slot(int xmode, int cfg, int mt, int rows) {
+// Tokens per TMA GEMV launch: up to this many tokens read the weights once in
+// one GEMV launch (on the MMA path from 2 tokens up); more go to the
+// tensor-core GEMM.
+constexpr int kGemvMaxTokens = 16;
+
+// Kernel of (mode, warps, tokens per launch, rows per block, MMA): one token
+// on 4, 8, 12 or 16 warps with dp4a or the MMA path, several tokens (MT = 2,
+// 4, 8, 16) on 8 or 16 warps with the MMA path, for int8 activations (xmode 0)
+// and, up to kFusedQuantMaxTokens tokens, bf16 activations quantised in the
+// kernel (xmode 1); row blocks of 32 or 16 rows.  Slot in the shared-memory
+// opt-in table, -1 if no such kernel.
+constexpr int kTmaNumSlots = 2 * 2 * 2 * kTmaNumCfg * 5;
+static_assert(kTmaNumSlots <= (int)(sizeof(DeviceInfo::tma_max_dyn) / sizeof(size_t)), "opt-in table");
+
+int tma_kernel_slot(int xmode, int cfg, int mt, int rows, int mma) {
     const int W = kTmaCfg[cfg][0];
-    const int base = rows == 16 ? 20 : 0;
-    if (mt == 1) return base + xmode * 10 + W / 4 - 1;
-    if (W != 8 && W != 16) return -1;
+    const int mti = mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : (mt == 8 ? 3 : (mt == 16 ? 4 : -1))));
+    if (mti < 0 || (mt > 1 && (!mma || (W != 8 && W != 16)))) return -1;
     if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
-    return base + xmode * 10 + 4 + 2 * (mt == 2 ? 0 : (mt == 4 ? 1 : 2)) + (W == 16 ? 1 : 0);
+    return (((xmode * 2 + (rows == 16 ? 1 : 0)) * 2 + (mma ? 1 : 0)) * kTmaNumCfg + cfg) * 5 + mti;
 }
 
-#define BITNET_TMA_VARIANTS(R)                                                                                   \
-    gemv_tma_kernel<0, 4, 1, R>, gemv_tma_kernel<0, 8, 1, R>, gemv_tma_kernel<0, 12, 1, R>,                     \
-        gemv_tma_kernel<0, 16, 1, R>, gemv_tma_kernel<0, 8, 2, R>, gemv_tma_kernel<0, 16, 2, R>,                \
-        gemv_tma_kernel<0, 8, 4, R>, gemv_tma_kernel<0, 16, 4, R>, gemv_tma_kernel<0, 8, 8, R>,                 \
-        gemv_tma_kernel<0, 16, 8, R>, gemv_tma_kernel<1, 4, 1, R>, gemv_tma_kernel<1, 8, 1, R>,                 \
-        gemv_tma_kernel<1, 12, 1, R>, gemv_tma_kernel<1, 16, 1, R>, gemv_tma_kernel<1, 8, 2, R>,                \
-        gemv_tma_kernel<1, 16, 2, R>, gemv_tma_kernel<1, 8, 4, R>, gemv_tma_kernel<1, 16, 4, R>,                \
-        nullptr, nullptr /* (bf16, 8 tokens): quantised beforehand instead */
-TmaKernel tma_kernel_for(int xmode, int cfg, int mt, int rows) {
-    static const TmaKernel table[40] = {BITNET_TMA_VARIANTS(32), BITNET_TMA_VARIANTS(16)};
-    const int slot = tma_kernel_slot(xmode, cfg, mt, rows);
-    return slot < 0 ? nullptr : table[slot];
+template <int X, int R, int MM>
+TmaKernel tma_kernel_w(int W, int mt) {
+    if (mt == 1) {
+        switch (W) {
+            case 4: return gemv_tma_kernel<X, 4, 1, R, MM>;
+            case 8: return gemv_tma_kernel<X, 8, 1, R, MM>;
+            case 12: return gemv_tma_kernel<X, 12, 1, R, MM>;
+            default: return gemv_tma_kernel<X, 16, 1, R, MM>;
+        }
+    }
+    if constexpr (MM == 1) {
+        const bool w16 = W == 16;
+        switch (mt) {
+            case 2: return w16 ? gemv_tma_kernel<X, 16, 2, R, 1> : gemv_tma_kernel<X, 8, 2, R, 1>;
+            case 4: return w16 ? gemv_tma_kernel<X, 16, 4, R, 1> : gemv_tma_kernel<X, 8, 4, R, 1>;
+            default: break;
+        }
+        if constexpr (X == 0) {
+            if (mt == 8) return w16 ? gemv_tma_kernel<0, 16, 8, R, 1> : gemv_tma_kernel<0, 8, 8, R, 1>;
+            if (mt == 16) return w16 ? gemv_tma_kernel<0, 16, 16, R, 1> : gemv_tma_kernel<0, 8, 16, R, 1>;
+        }
+    }
+    return nullptr;
 }
-#undef BITNET_TMA_VARIANTS
+
+template <int X, int R>
+TmaKernel tma_kernel_m(int W, int mt, int mma) {
+    return mma ? tma_kernel_w<X, R, 1>(W, mt) : tma_kernel_w<X, R, 0>(W, mt);
+}
+
+TmaKernel tma_kernel_for(int xmode, int cfg, int mt, int rows, int mma) {
+    if (tma_kernel_slot(xmode, cfg, mt, rows, mma) < 0) return nullptr;
+    const int W = kTmaCfg[cfg][0];
+    if (xmode == 0) return rows == 16 ? tma_kernel_m<0, 16>(W, mt, mma) : tma_kernel_m<0, 32>(W, mt, mma);
+    return rows == 16 ? tma_kernel_m<1, 16>(W, mt, mma) : tma_kernel_m<1, 32>(W, mt, mma);
+}
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int rows) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int rows, int mma) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    const int si = tma_kernel_slot(xmode, cfg, mt, rows);
+    const int si = tma_kernel_slot(xmode, cfg, mt, rows, mma);
     if (si < 0) return 0;
     size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, cfg, mt, rows);
+        TmaKernel kern = tma_kernel_for(xmode, cfg, mt, rows, mma);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -378,8 +407,9 @@ struct TmaPlan {
     bool use;
     int cfg, slices, max_blocks, grid;
     int ns;            // ring depth per warp
-    int mt;            // tokens per launch (1, 2, 4, 8)
+    int mt;            // tokens per launch (1, 2, 4, 8, 16)
     int rows;          // rows per block (32 or 16)
+    int mma;           // 1: the MMA product, 0: dp4a (one token only)
     int64_t nblocks;
     size_t smem;
     int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
@@ -392,17 +422,18 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     const GemvTune &tn = gemv_tune();
     TmaPlan p{};
     const int tune = tn.tma;
-    if (M < 1 || M > 8 || tune == 0 || K < kTmaSliceK || N < 1) return p;
+    if (M < 1 || M > kGemvMaxTokens || tune == 0 || K < kTmaSliceK || N < 1) return p;
     // a lane accumulates one row's whole K: |acc_j| <= 4096 * K_pad stays
     // inside int32 for K_pad <= 2^19 (shared memory caps K lower still)
     if (k_pad(K) > ((int64_t)1 << 19)) return p;
-    p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
+    p.mt = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : (M <= 8 ? 8 : 16)));
+    p.mma = p.mt > 1 ? 1 : (tn.mma == 1 ? 1 : 0);
     const int64_t row_bytes = packed_row_bytes(K);
     // co-residency mode (tuning field `cores` = 1, see above); eight tokens
     // keep 32-row blocks: their 16-warp variant has no registers to spare for
     // the second lane of a row
     const bool cores = tn.cores == 1;
-    p.rows = (!cores || ceil_div(N, kTmaRows) >= kRefSMs || p.mt == 8) ? 32 : 16;
+    p.rows = (!cores || ceil_div(N, kTmaRows) >= kRefSMs || p.mt >= 8) ? 32 : 16;
     if (tn.rows == 16 || tn.rows == 32) p.rows = tn.rows;
     p.nblocks = ceil_div(N, p.rows);
     p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
@@ -434,9 +465,10 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
                     const TmaPlan &tp, cudaStream_t st) {
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt, tp.rows);
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt, tp.rows, tp.mma);
     if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
-    if (tensor_map_encoder() == nullptr || tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt, tp.rows))
+    if (tensor_map_encoder() == nullptr ||
+        tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt, tp.rows, tp.mma))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;
@@ -790,7 +822,7 @@ struct GemmPlan {
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinear) {
     GemmPlan p{};
     (void)q_tma_ok;
-    if (M <= 8) {  // decode and small batches: the TMA GEMV reads the weights once
+    if (M <= kGemvMaxTokens) {  // decode and small batches: the TMA GEMV reads the weights once
         const TmaPlan tp = tma_plan(M, N, K);
         if (tp.use) {
             p.path = kPathGemv;
@@ -984,7 +1016,7 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    if (p.path == kPathGemv && M > kFusedQuantMaxTokens && M <= 8 && tma_plan(M, N, K).use) {
+    if (p.path == kPathGemv && M > kFusedQuantMaxTokens && M <= kGemvMaxTokens && tma_plan(M, N, K).use) {
         // small batch: quantise the tokens once, then one pass over the weights
         int8_t *q = static_cast<int8_t *>(workspace);
         float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * K, 256));

@@ -1,17 +1,16 @@
-// gemv_tma.cuh -- the decode GEMV (one to eight tokens): packed weights stream
-// through shared memory by TMA, one row per lane.
+// gemv_tma.cuh -- the decode GEMV (one to sixteen tokens): packed weights
+// stream through shared memory by TMA.
 //
-// Same contraction and decode as gemv.cuh (layout v1 words, shift-free dp4a
-// on codes scaled by 4^j, activation-sum correction); what differs is how the
-// weights reach the lanes:
+// Same contraction and decode as gemv.cuh (layout v1 words, codes scaled by
+// 4^j, activation-sum correction); what differs is how the weights reach the
+// lanes:
 //   - The packed matrix is a 2-D byte tensor [N rows, K_pad/4 bytes].  A TMA
-//     box is ROWS rows x 128 bytes (512 k): 32 rows (4 KB, one lane per row)
-//     or 16 rows (2 KB, two lanes per row, each taking half of the row's 8
-//     chunks), written to shared memory with the 128-byte swizzle, so a lane
-//     reading 16-byte chunk c of box row r (address r*128 + ((c ^ (r & 7)) *
-//     16)) is free of bank conflicts.  16-row blocks give shapes of fewer than
-//     148 32-row blocks one block for every SM.
-//   - Work items are (32-row block, 128-byte K-slice) pairs.  CTA b owns row
+//     box is ROWS rows x 128 bytes (512 k): 32 rows (4 KB) or 16 rows (2 KB),
+//     written to shared memory with the 128-byte swizzle (16-byte unit u of
+//     box row r at r*128 + ((u ^ (r & 7)) * 16)), so that the reads below are
+//     free of bank conflicts.  16-row blocks give shapes of fewer than 148
+//     32-row blocks one block for every SM.
+//   - Work items are (row block, 128-byte K-slice) pairs.  CTA b owns row
 //     blocks b, b + gridDim.x, ...; its items, in (row block, slice) order, are
 //     split into equal contiguous ranges, one per warp, which keeps every warp
 //     busy for any K and makes a warp leave a row block at most a few times.
@@ -19,14 +18,18 @@
 //     lane 0 issues the TMA for the item NS ahead as soon as the warp has read
 //     a stage, so up to NS boxes per warp are in flight without holding
 //     registers.
-//   - Activations live in shared memory as one linear array per token; all
-//     lanes read the same 16 bytes at a time (a broadcast).  With several
-//     tokens (MT = 2, 4, 8) every weight box is still read from HBM once: the
-//     four code masks of each word are computed once and reused per token.
+//   - Activations live in shared memory as one linear array per token, staged
+//     with all of a thread's loads in flight at once.
+//   - The product: for one token, each lane takes one row (or half of one)
+//     and dots its 16-byte chunks against the activations (all lanes read the
+//     same 16 bytes: a broadcast) with dp4a; for 2..16 tokens (and, as a
+//     tuned option, for one), the warp runs m16n8k32 integer MMAs over the box
+//     (see gemv_tma_kernel), so that every weight box is read from HBM once
+//     and the instruction count per box hardly grows with the tokens.
 //   - A warp adds its per-row partial sums into a per-row-block int32
 //     accumulator in shared memory (atomics: exact and order-free) whenever its
 //     item sequence leaves a row block; the warp whose contribution completes
-//     the block's item count writes the 32 results.
+//     the block's item count writes the results.
 //   - Every mbarrier wait is bounded in time.  A warp that gives up records
 //     BITNET_ERR_DEVICE_TIMEOUT, waits (bounded) for its own boxes in flight and
 //     stops; that row block's outputs are then left unwritten.
@@ -67,10 +70,14 @@ struct GemvTmaArgs {
 // Dynamic shared memory of a launch: ring of warps x stages boxes of `rows`
 // rows, linear activations, per-row-block accumulators and counters, slice
 // sums, mbarriers.
+__host__ __device__ inline int64_t gemv_tma_token_stride(int slices, int tokens) {
+    return (int64_t)slices * kTmaSliceK + (tokens > 1 ? 64 : 0);
+}
+
 __host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int slices, int max_blocks_cta,
                                                       int tokens = 1, int rows = kTmaRows) {
     return 1024 /* alignment slack */ + (size_t)warps * stages * rows * kTmaSliceBytes +
-           (size_t)tokens * slices * kTmaSliceK + (size_t)max_blocks_cta * tokens * rows * 4 +
+           (size_t)tokens * gemv_tma_token_stride(slices, tokens) + (size_t)max_blocks_cta * tokens * rows * 4 +
            (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
 }
 
@@ -146,77 +153,118 @@ __device__ __forceinline__ void slice_sum(int *qslice, int64_t p, const uint4 &v
     if ((threadIdx.x & 31) == 0) qslice[p >> 5] = t;
 }
 
-// Linear staging of int8 activations: qlin[k] = q[k] for k < K, 0 up to kq
-// (kq a multiple of 512), with the sum of every 512-k slice in qslice.
-__device__ __forceinline__ void stage_qlin_int8(int8_t *qlin, int *qslice, const int8_t *qrow, int64_t K,
-                                                int64_t kq) {
-    const bool vec = ((reinterpret_cast<uintptr_t>(qrow) & 15) == 0);
-    for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
-        const int64_t k0 = p * 16;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (vec && k0 + 16 <= K) {
-            v = *reinterpret_cast<const uint4 *>(qrow + k0);
-        } else if (k0 < K) {
-            uint32_t w[4] = {0u, 0u, 0u, 0u};
-            for (int t = 0; t < 16 && k0 + t < K; ++t) w[t >> 2] |= (uint32_t)(uint8_t)qrow[k0 + t] << (8 * (t & 3));
-            v = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        *reinterpret_cast<uint4 *>(qlin + k0) = v;
-        slice_sum(qslice, p, v);
-    }
-}
+// Pieces of 16 k a thread keeps in registers while staging: their loads are
+// issued together, one memory round trip for all of them (a thread takes
+// pieces threadIdx.x + i * blockDim.x, so a CTA of 512 threads stages 2048
+// pieces, four 32 K-long rows or one of 32 K, per round trip).
+constexpr int kStageHeld = 4;
 
-// Linear staging with fused per-token quantisation of bf16 activations (same
-// arithmetic as quant_act_kernel<>), slice sums as above.  Returns the scale.
-__device__ __forceinline__ float stage_qlin_bf16(int8_t *qlin, int *qslice, float *red, const uint16_t *xrow,
-                                                 int64_t K, int64_t kq) {
-    const bool vec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
-    const int64_t npieces = ceil_div(K, 16);
-    float amax = 0.0f;
-    for (int64_t p = threadIdx.x; p < npieces; p += blockDim.x) {
-        uint4 lo, hi;
-        load_x16(xrow, K, p, vec, lo, hi);
-        amax = amax16(lo, hi, amax);
-    }
-    amax = block_reduce(amax, [](float u, float v) { return fmaxf(u, v); }, red);
-    const float sc = __fdiv_rn(127.0f, amax > kQuantEps ? amax : kQuantEps);
-    for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (p < npieces) {
-            uint4 lo, hi;
-            load_x16(xrow, K, p, vec, lo, hi);
-            quant16(lo, hi, sc, v);
-        }
-        *reinterpret_cast<uint4 *>(qlin + p * 16) = v;
-        slice_sum(qslice, p, v);
-    }
-    return sc;
-}
-
-// Linear staging with fused quantisation of MT tokens at once (same
-// arithmetic as quant_act_kernel<>): one pass over every token's row for the
-// absmax values, one block reduction for all of them, then every token is
-// quantised, with slice sums as above.  Token slots t >= M are staged as
-// zeros.  `red` holds MT x 32 floats.
+// Cursor over a thread's pieces of the flat (token, piece) order, ppt pieces
+// per token, stepping by blockDim.x without a division per step.
 template <int MT>
-__device__ __forceinline__ void stage_qlin_bf16_tokens(int8_t *qlin, int *qslice, int slices, float *red,
-                                                       const uint16_t *x, int M, int64_t K, int64_t kq,
-                                                       float (&sc)[MT]) {
-    const int64_t npieces = ceil_div(K, 16);
+struct PieceCursor {
+    int t, pp, qb, rb, ppt;
+    __device__ __forceinline__ explicit PieceCursor(int ppt_) : ppt(ppt_) {
+        if (MT == 1) {
+            t = 0, pp = threadIdx.x, qb = 0, rb = blockDim.x;
+        } else {
+            t = threadIdx.x / ppt, pp = threadIdx.x - t * ppt;
+            qb = blockDim.x / ppt, rb = blockDim.x - qb * ppt;
+        }
+    }
+    __device__ __forceinline__ bool valid() const { return MT == 1 ? pp < ppt : t < MT; }
+    __device__ __forceinline__ void next() {
+        pp += rb;
+        if (MT > 1) {
+            t += qb;
+            if (pp >= ppt) pp -= ppt, ++t;
+        }
+    }
+};
+
+// Staging of int8 activations for MT token slots: qlin[t * ldx + k] = q[t * K
+// + k] for t < M and k < K, 0 elsewhere up to kq (a multiple of 512), with
+// the sum of every 512-k slice of token t in qslice[t * slices + j].  Piece p
+// (16 k) of the flat (token, piece) order is staged by thread p mod blockDim.x;
+// a warp takes 32 consecutive pieces, one slice of one token, so one warp
+// reduction gives the slice's sum.
+template <int MT>
+__device__ __forceinline__ void stage_tokens_int8(int8_t *qlin, int64_t ldx, int *qslice, int slices, const int8_t *q,
+                                                  int M, int64_t K, int64_t kq) {
+    PieceCursor<MT> cur((int)(kq / 16));  // ppt and blockDim.x are multiples of 32
+    while (cur.valid()) {
+        uint4 v[kStageHeld];
+        int ts[kStageHeld], ps[kStageHeld];
+#pragma unroll
+        for (int i = 0; i < kStageHeld; ++i) {
+            ts[i] = cur.valid() ? cur.t : MT, ps[i] = cur.pp;
+            v[i] = make_uint4(0u, 0u, 0u, 0u);
+            const int64_t k0 = (int64_t)ps[i] * 16;
+            if (ts[i] < M && k0 < K) {
+                const int8_t *qrow = q + (int64_t)ts[i] * K;
+                if ((reinterpret_cast<uintptr_t>(qrow) & 15) == 0 && k0 + 16 <= K) {
+                    v[i] = *reinterpret_cast<const uint4 *>(qrow + k0);
+                } else {
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    for (int b = 0; b < 16 && k0 + b < K; ++b) w[b >> 2] |= (uint32_t)(uint8_t)qrow[k0 + b] << (8 * (b & 3));
+                    v[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            cur.next();
+        }
+#pragma unroll
+        for (int i = 0; i < kStageHeld; ++i) {
+            if (ts[i] < MT) {  // warp-uniform
+                *reinterpret_cast<uint4 *>(qlin + ts[i] * ldx + (int64_t)ps[i] * 16) = v[i];
+                slice_sum(qslice + ts[i] * slices, ps[i], v[i]);
+            }
+        }
+    }
+}
+
+// Staging with fused per-token quantisation of bf16 activations (the same
+// arithmetic as quant_act_kernel<>): every token's absmax over one pass that
+// keeps the first kStageHeld pieces per thread in registers (loads issued
+// together), one block reduction for all tokens, then the codes, with slice
+// sums as above.  Pieces beyond those held are read again.  Returns the
+// scales in sc; token slots t >= M are staged as zeros.  `red` holds MT x 32
+// floats.
+template <int MT>
+__device__ __forceinline__ void stage_tokens_bf16(int8_t *qlin, int64_t ldx, int *qslice, int slices, float *red,
+                                                  const uint16_t *x, int M, int64_t K, int64_t kq, float (&sc)[MT]) {
+    const int ppt = (int)(kq / 16);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    auto load = [&](int t, int pp, uint4 &lo, uint4 &hi) {
+        lo = hi = make_uint4(0u, 0u, 0u, 0u);
+        if (t < M) {
+            const uint16_t *xr = x + (int64_t)t * K;
+            load_x16(xr, K, pp, (reinterpret_cast<uintptr_t>(xr) & 15) == 0, lo, hi);
+        }
+    };
     float am[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) am[t] = 0.0f;
-    for (int64_t p = threadIdx.x; p < npieces; p += blockDim.x) {
+    auto amax_into = [&](int t, const uint4 &lo, const uint4 &hi) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            if (t < M) {
-                const uint16_t *xr = x + (int64_t)t * K;
-                uint4 lo, hi;
-                load_x16(xr, K, p, (reinterpret_cast<uintptr_t>(xr) & 15) == 0, lo, hi);
-                am[t] = amax16(lo, hi, am[t]);
-            }
-        }
+        for (int u = 0; u < MT; ++u)
+            if (u == t) am[u] = amax16(lo, hi, am[u]);
+    };
+    PieceCursor<MT> cur(ppt);
+    uint4 held[kStageHeld][2];
+    int ts[kStageHeld], ps[kStageHeld];
+#pragma unroll
+    for (int i = 0; i < kStageHeld; ++i) {
+        ts[i] = cur.valid() ? cur.t : MT, ps[i] = cur.pp;
+        load(ts[i], ps[i], held[i][0], held[i][1]);
+        cur.next();
+    }
+#pragma unroll
+    for (int i = 0; i < kStageHeld; ++i) amax_into(ts[i], held[i][0], held[i][1]);
+    PieceCursor<MT> rest = cur;
+    for (; cur.valid(); cur.next()) {
+        uint4 lo, hi;
+        load(cur.t, cur.pp, lo, hi);
+        amax_into(cur.t, lo, hi);
     }
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
@@ -232,40 +280,76 @@ __device__ __forceinline__ void stage_qlin_bf16_tokens(int8_t *qlin, int *qslice
         for (int w = 0; w < nwarps; ++w) v = fmaxf(v, red[t * 32 + w]);
         sc[t] = t < M ? __fdiv_rn(127.0f, v > kQuantEps ? v : kQuantEps) : 0.0f;
     }
+    auto put = [&](int t, int pp, const uint4 &lo, const uint4 &hi) {  // t < MT: warp-uniform
+        float s = sc[0];
 #pragma unroll
-    for (int t = 0; t < MT; ++t) {
-        const uint16_t *xr = x + (int64_t)t * K;
-        const bool vec = (reinterpret_cast<uintptr_t>(xr) & 15) == 0;
-        for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < M && p < npieces) {
-                uint4 lo, hi;
-                load_x16(xr, K, p, vec, lo, hi);
-                quant16(lo, hi, sc[t], v);
-            }
-            *reinterpret_cast<uint4 *>(qlin + t * kq + p * 16) = v;
-            slice_sum(qslice + t * slices, p, v);
-        }
+        for (int u = 1; u < MT; ++u)
+            if (u == t) s = sc[u];
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (t < M) quant16(lo, hi, s, v);
+        *reinterpret_cast<uint4 *>(qlin + t * ldx + (int64_t)pp * 16) = v;
+        slice_sum(qslice + t * slices, pp, v);
+    };
+#pragma unroll
+    for (int i = 0; i < kStageHeld; ++i)
+        if (ts[i] < MT) put(ts[i], ps[i], held[i][0], held[i][1]);
+    for (; rest.valid(); rest.next()) {
+        uint4 lo, hi;
+        load(rest.t, rest.pp, lo, hi);
+        put(rest.t, rest.pp, lo, hi);
     }
 }
 
 // ------------------------------------------------------------------ kernel
 
-// Resident CTAs the register budget leaves room for: two for every variant of
-// up to two tokens and for the 8-warp ones of up to four, so that the next
-// launch's CTA can start beside this one's on an SM (and request its weights)
-// while this launch finishes there.
-template <int W, int MT>
-constexpr int gemv_tma_min_blocks() { return (MT <= 2 || (W <= 8 && MT <= 4)) ? 2 : 1; }
+// One m16n8k32 integer MMA on the warp's tensor-core path: A unsigned bytes
+// (scaled 2-bit codes), B signed int8 activations, exact int32 accumulation.
+// Fragments (PTX ISA, mma.m16n8k32 with 8-bit operands; g = lane / 4, t =
+// lane % 4): a0 = A[g][4t..4t+3], a1 = A[g+8][4t..], a2 = A[g][16+4t..], a3 =
+// A[g+8][16+4t..]; b0 = B[4t..4t+3][g], b1 = B[16+4t..][g]; d0,d1 = D[g][2t,
+// 2t+1], d2,d3 = D[g+8][2t, 2t+1].
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-template <int XMODE, int W, int MT, int ROWS>
-__global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
+// Resident CTAs the register budget leaves room for: two for the dp4a
+// variants of up to two tokens and for the 8-warp ones of up to four, so that
+// the next launch's CTA can start beside this one's on an SM (and request its
+// weights) while this launch finishes there; one for the MMA variants, whose
+// accumulators take 32 registers per 8 tokens.
+template <int W, int MT, int MMA>
+constexpr int gemv_tma_min_blocks() { return MMA ? 1 : ((MT <= 2 || (W <= 8 && MT <= 4)) ? 2 : 1); }
+
+// MMA = 0: every lane dots its row's 16-byte chunks against the activations
+// with dp4a (one token).  MMA = 1: the warp multiplies the box with m16n8k32
+// integer MMAs, 16 rows x 8 tokens x 32 k at a time, for 1 to 16 tokens:
+//   - A is one code plane of the packed words: (word & (3 << 2j)) holds the
+//     codes of k = 16 w + 4 j + b (byte b) times 4^j, as unsigned bytes; the
+//     four planes accumulate apart and are scaled back (exact shifts) at the
+//     flush, as in the dp4a path.
+//   - The MMA's k index is any order both operands agree on: lane (g, t) of a
+//     128-k chunk c takes word t of the chunk's first 16-byte unit (a0, a1) and
+//     word t of its second unit (a2, a3), for rows g and g + 8; its B
+//     registers are then the activation bytes 128 c + 16 t + 4 j .. + 3 and
+//     that + 64, i.e. one 16-byte load gives b0 (or b1) for all four planes.
+//   - Token rows sit ldx = kq + 64 bytes apart, so that the eight tokens' loads
+//     of a quarter warp fall in distinct banks; the box rows' loads are
+//     conflict-free under the 128-byte swizzle (distinct units per row).
+template <int XMODE, int W, int MT, int ROWS, int MMA>
+__global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
-    static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8, "tokens per launch");
+    static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8 || MT == 16, "tokens per launch");
+    static_assert(MMA || MT == 1, "several tokens take the MMA path");
     static_assert(ROWS == 32 || ROWS == 16, "rows per box");
-    constexpr int kLPR = kTmaRows / ROWS;               // lanes per row
-    constexpr int kCPL = 8 / kLPR;                      // 16-byte chunks per lane per box
+    constexpr int kLPR = kTmaRows / ROWS;               // lanes per row (output stores; dp4a MAC)
+    constexpr int kCPL = 8 / kLPR;                      // 16-byte chunks per lane per box (dp4a)
     constexpr int kBoxBytes = ROWS * kTmaSliceBytes;
+    constexpr int kRG = ROWS / 16;                      // 16-row MMA groups per box
+    constexpr int kNT = (MT + 7) / 8;                   // 8-token MMA tiles
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ float red[(XMODE == 1 ? MT : 1) * 32];
@@ -274,13 +358,14 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     const int ns = a.ns, slices = a.slices;
     const int64_t cid = blockIdx.x, ncl = gridDim.x;  // row blocks cid, cid + ncl, ...
     const int64_t kq = (int64_t)slices * kTmaSliceK;
+    const int64_t ldx = gemv_tma_token_stride(slices, MT);
 
     // 1024-byte alignment of the ring (the 128-byte swizzle repeats every 8
     // rows of 128 bytes), computed on the shared-window address so that every
     // pointer below stays a shared-memory pointer
     uint8_t *ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kBoxBytes);      // [MT][kq]
-    int *accs = reinterpret_cast<int *>(qlin + MT * kq);                       // [slot][MT][ROWS]
+    int8_t *qlin = reinterpret_cast<int8_t *>(ring + W * ns * kBoxBytes);      // [MT][ldx]
+    int *accs = reinterpret_cast<int *>(qlin + MT * ldx);                      // [slot][MT][ROWS]
     int *done = accs + a.max_blocks_cta * MT * ROWS;                           // [slot] items done
     int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
     uint64_t *bars =
@@ -288,6 +373,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int brow = lane / kLPR, part = lane % kLPR;  // this lane's box row and chunk half
+    const int mg = lane >> 2, mt4 = lane & 3;          // MMA fragment coordinates (g, t)
     // this CTA's items, in (row block, slice) order
     const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
     const int64_t items = nb_cta * slices;
@@ -333,23 +419,12 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
     pdl_wait();
 
     float sc[MT];
-    if (XMODE == 1 && MT > 1) stage_qlin_bf16_tokens<MT>(qlin, qslice, slices, red, a.x, a.M, a.K, kq, sc);
+    if (XMODE == 0) {
+        stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq);
 #pragma unroll
-    for (int t = 0; t < MT; ++t) {
-        if (XMODE == 1 && MT > 1) break;  // staged above
-        sc[t] = 0.0f;
-        int8_t *qt = qlin + t * kq;
-        int *qst = qslice + t * slices;
-        if (t < a.M) {
-            if (XMODE == 0)
-                stage_qlin_int8(qt, qst, a.q + (int64_t)t * a.K, a.K, kq);
-            else
-                sc[t] = stage_qlin_bf16(qt, qst, red, a.x + (int64_t)t * a.K, a.K, kq);
-        } else {  // unused token slot: zeros, contributes nothing and is not stored
-            for (int64_t p = threadIdx.x; p < kq / 16; p += blockDim.x)
-                reinterpret_cast<uint4 *>(qt)[p] = make_uint4(0u, 0u, 0u, 0u);
-            for (int j = threadIdx.x; j < slices; j += blockDim.x) qst[j] = 0;
-        }
+        for (int t = 0; t < MT; ++t) sc[t] = 0.0f;
+    } else {
+        stage_tokens_bf16<MT>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
     }
     __syncthreads();
     float f[MT];
@@ -359,19 +434,52 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
         if (t < a.M && a.y_bf16 != nullptr) f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
     }
 
-    int acc[MT][4], corr[MT];
+    // dp4a accumulators: one row (or half of one), per code plane
+    int acc[4] = {0, 0, 0, 0}, corr = 0;
+    // MMA accumulators: [token tile][row group][code plane] fragments, and the
+    // activation-sum correction of this lane's two tokens per tile
+    int macc[MMA ? kNT : 1][MMA ? kRG : 1][4][4];
+    int mcorr[MMA ? kNT : 1][2];
+    auto zero_acc = [&]() {
+        acc[0] = acc[1] = acc[2] = acc[3] = corr = 0;
+        if (MMA) {
 #pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
+            for (int nt = 0; nt < kNT; ++nt) {
+                mcorr[nt][0] = mcorr[nt][1] = 0;
+#pragma unroll
+                for (int rg = 0; rg < kRG; ++rg)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) macc[nt][rg][j][0] = macc[nt][rg][j][1] = macc[nt][rg][j][2] = macc[nt][rg][j][3] = 0;
+            }
+        }
+    };
+    zero_acc();
     int ncontrib = 0;
     // folds this warp's partial sums of slot `sl` into shared memory (the
-    // lanes sharing a row each add their half; the activation-sum correction
-    // is taken once per row); the warp completing the slot's items writes its
-    // results
+    // activation-sum correction is taken once per row and token); the warp
+    // completing the slot's items writes its results
     auto flush = [&](int sl) {
+        if (MMA) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            const int v = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) - (part == 0 ? corr[t] : 0);
-            atomicAdd(&accs[(sl * MT + t) * ROWS + brow], v);
+            for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = nt * 8 + 2 * mt4 + e;
+                    if (tok < MT) {
+#pragma unroll
+                        for (int rg = 0; rg < kRG; ++rg)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int (&m)[4][4] = macc[nt][rg];
+                                const int v = m[0][2 * h + e] + (m[1][2 * h + e] >> 2) + (m[2][2 * h + e] >> 4) +
+                                              (m[3][2 * h + e] >> 6) - mcorr[nt][e];
+                                atomicAdd(&accs[(sl * MT + tok) * ROWS + rg * 16 + h * 8 + mg], v);
+                            }
+                    }
+                }
+        } else {
+            const int v = acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6) - (part == 0 ? corr : 0);
+            atomicAdd(&accs[sl * ROWS + brow], v);
         }
         __threadfence_block();
         __syncwarp();
@@ -392,8 +500,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
                 }
             }
         }
-#pragma unroll
-        for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = corr[t] = 0;
+        zero_acc();
         ncontrib = 0;
     };
 
@@ -409,47 +516,66 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT>())
                 mbar_wait_bounded(&mybar[(n + d) % ns], (uint32_t)((n + d) / ns) & 1u);
             break;
         }
-        const uint8_t *row = myring + s * kBoxBytes + brow * kTmaSliceBytes;
-        const int8_t *qk = qlin + cj * kTmaSliceK;
+        if (MMA) {
+            const uint8_t *box = myring + s * kBoxBytes + mg * kTmaSliceBytes + 4 * mt4;
+            const int8_t *xs = qlin + cj * kTmaSliceK + 16 * mt4;
 #pragma unroll
-        for (int cc = 0; cc < kCPL; ++cc) {
-            const int c = part * kCPL + cc;
-            const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (brow & 7)) << 4));
-            if (MT == 1) {
-                const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
-                const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];
-                mac_word(acc[0], w.x, x0);
-                mac_word(acc[0], w.y, x1);
-                mac_word(acc[0], w.z, x2);
-                mac_word(acc[0], w.w, x3);
-            } else {
-                // the four scaled code masks of each word, shared by all tokens
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                uint32_t mk[4][4];
+            for (int c = 0; c < 4; ++c) {  // 128-k chunks of the slice
+                uint32_t bl[kNT][4], bh[kNT][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    mk[i][0] = ww[i] & 0x03030303u;
-                    mk[i][1] = ww[i] & 0x0C0C0C0Cu;
-                    mk[i][2] = ww[i] & 0x30303030u;
-                    mk[i][3] = ww[i] & 0xC0C0C0C0u;
+                for (int nt = 0; nt < kNT; ++nt) {
+                    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+                    const int tok = nt * 8 + mg;
+                    if (tok < MT) {
+                        const int8_t *xp = xs + tok * ldx + 128 * c;
+                        v0 = *reinterpret_cast<const uint4 *>(xp);
+                        v1 = *reinterpret_cast<const uint4 *>(xp + 64);
+                    }
+                    bl[nt][0] = v0.x, bl[nt][1] = v0.y, bl[nt][2] = v0.z, bl[nt][3] = v0.w;
+                    bh[nt][0] = v1.x, bh[nt][1] = v1.y, bh[nt][2] = v1.z, bh[nt][3] = v1.w;
                 }
+                // rows mg and mg + 8 of each group share (row & 7) = mg
+                const int u0 = ((2 * c) ^ mg) << 4, u1 = ((2 * c + 1) ^ mg) << 4;
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    const uint4 *qp = reinterpret_cast<const uint4 *>(qk + t * kq + c * 64);
+                for (int rg = 0; rg < kRG; ++rg) {
+                    const uint8_t *r0 = box + rg * 16 * kTmaSliceBytes, *r1 = r0 + 8 * kTmaSliceBytes;
+                    const uint32_t w00 = *reinterpret_cast<const uint32_t *>(r0 + u0);
+                    const uint32_t w01 = *reinterpret_cast<const uint32_t *>(r0 + u1);
+                    const uint32_t w10 = *reinterpret_cast<const uint32_t *>(r1 + u0);
+                    const uint32_t w11 = *reinterpret_cast<const uint32_t *>(r1 + u1);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 x = qp[i];
-                        acc[t][0] = dp4a_us(mk[i][0], x.x, acc[t][0]);
-                        acc[t][1] = dp4a_us(mk[i][1], x.y, acc[t][1]);
-                        acc[t][2] = dp4a_us(mk[i][2], x.z, acc[t][2]);
-                        acc[t][3] = dp4a_us(mk[i][3], x.w, acc[t][3]);
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t mk = 0x03030303u << (2 * j);
+#pragma unroll
+                        for (int nt = 0; nt < kNT; ++nt)
+                            mma_u8s8(macc[nt][rg][j], w00 & mk, w10 & mk, w01 & mk, w11 & mk, bl[nt][j], bh[nt][j]);
                     }
                 }
             }
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = nt * 8 + 2 * mt4 + e;
+                    if (tok < MT) mcorr[nt][e] += qslice[tok * slices + cj];
+                }
+        } else {
+            const uint8_t *row = myring + s * kBoxBytes + brow * kTmaSliceBytes;
+            const int8_t *qk = qlin + cj * kTmaSliceK;
+#pragma unroll
+            for (int cc = 0; cc < kCPL; ++cc) {
+                const int c = part * kCPL + cc;
+                const uint4 w = *reinterpret_cast<const uint4 *>(row + ((c ^ (brow & 7)) << 4));
+                const uint4 *qp = reinterpret_cast<const uint4 *>(qk + c * 64);
+                const uint4 x0 = qp[0], x1 = qp[1], x2 = qp[2], x3 = qp[3];
+                mac_word(acc, w.x, x0);
+                mac_word(acc, w.y, x1);
+                mac_word(acc, w.z, x2);
+                mac_word(acc, w.w, x3);
+            }
+            corr += qslice[cj];
         }
         ++ncontrib;
-#pragma unroll
-        for (int t = 0; t < MT; ++t) corr[t] += qslice[t * slices + cj];
         __syncwarp();
         if (lane == 0 && n + ns < n_items) issue_next(s);
         if (++s == ns) {

@@ -1,6 +1,6 @@
-"""Parity of the small-batch decode (2..8 tokens through the TMA-staged GEMV,
-every weight box read once for all tokens): int32 and BitLinear outputs on
-ragged shapes and token counts that leave unused token slots."""
+"""Parity of the small-batch decode (2..16 tokens through the TMA-staged GEMV's
+MMA product, every weight box read once for all tokens): int32 and BitLinear
+outputs on ragged shapes and token counts that leave unused token slots."""
 import numpy as np
 import pytest
 
@@ -24,7 +24,8 @@ def _cuda():
 
 
 @pytest.mark.parametrize("M,N,K", [(2, 1000, 2560), (3, 33, 700), (4, 257, 1024), (5, 300, 5120), (7, 64, 3200),
-                                   (8, 2560, 6912), (6, 13824, 2560)])
+                                   (8, 2560, 6912), (6, 13824, 2560), (9, 300, 2560), (13, 33, 700),
+                                   (12, 2560, 6912), (16, 13824, 2560), (16, 5120, 3200)])
 def test_small_batch_int32_exact(M, N, K):
     q, w = synth.uniform_int8_ternary(N, K, seed=M * 1000 + N + K, M=M)
     q[-1, :7] = -128
@@ -32,10 +33,10 @@ def test_small_batch_int32_exact(M, N, K):
     assert np.array_equal(y.cpu().numpy(), oracle.gemm_i32(q, w))
 
 
-# 2..4 tokens are quantised inside the GEMV prologue, 5..8 in a pass of their
+# 2..4 tokens are quantised inside the GEMV prologue, 5..16 in a pass of their
 # own first: both sides of that boundary are here
 @pytest.mark.parametrize("M,N,K", [(2, 500, 2560), (3, 6912, 2560), (4, 257, 1536), (5, 300, 3200),
-                                   (8, 2560, 6912)])
+                                   (8, 2560, 6912), (11, 300, 3200), (16, 2560, 6912)])
 def test_small_batch_bitlinear(M, N, K):
     x, W = synth.bitlinear_inputs(M, N, K, seed=M)
     x[1] = 0  # a zero token among them
@@ -54,12 +55,12 @@ def test_small_batch_bitlinear(M, N, K):
 def test_bitlinear_same_bits_on_every_path():
     """A token's bf16 output does not depend on which path quantised it: the
     single-token prologue (1 token), the multi-token prologue (2..4), a
-    quantisation pass before the GEMV (5..8) or before the tensor-core GEMM (9
-    and more).  All of them take the scale and the codes with the same fp32
+    quantisation pass before the GEMV (5..16) or before the tensor-core GEMM
+    (17 and more).  All of them take the scale and the codes with the same fp32
     operations and rescale the same way, so the shared tokens' outputs must be
     identical bit for bit (a one-ulp scale difference would change codes)."""
     N, K = 300, 2560
-    x, W = synth.bitlinear_inputs(12, N, K, seed=5)
+    x, W = synth.bitlinear_inputs(20, N, K, seed=5)
     x[7, :] = 0
     g = oracle.absmean(W)
     wt = oracle.ternarize(W, g)
@@ -67,10 +68,10 @@ def test_bitlinear_same_bits_on_every_path():
     gamma = torch.tensor([float(g)], dtype=torch.float32, device="cuda")
     xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
     outs = {M: bn.bitnet_bitlinear(xd[:M].contiguous(), packed, gamma, N).view(torch.int16).cpu().numpy()
-            for M in (1, 2, 3, 4, 5, 8, 9, 12)}
-    full = outs[12]
+            for M in (1, 2, 3, 4, 5, 8, 9, 12, 16, 17, 20)}
+    full = outs[20]
     for M, y in outs.items():
-        assert np.array_equal(y, full[:M]), f"{M} tokens: bf16 bits differ from the 12-token run"
+        assert np.array_equal(y, full[:M]), f"{M} tokens: bf16 bits differ from the 20-token run"
     y_ref = oracle.bitlinear(x, wt, g)[0]
     yf = torch.from_numpy(full).view(torch.bfloat16).float().numpy().astype(np.float64)
     err = np.abs(yf - y_ref)

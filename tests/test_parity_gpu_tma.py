@@ -3,8 +3,8 @@
 A child process forces the variant (BITNET_GEMV_TUNE, read once per process:
 warps per CTA, ring depth, CTAs per SM) on shapes with ragged row blocks (N
 not a multiple of 32), partial K-slices (K_pad/4 not a multiple of 128), a
-single row block, several row blocks per CTA, and 1, 3 or 8 tokens; int32 and
-BitLinear outputs.
+single row block, several row blocks per CTA, and 1, 3, 8 or 13 tokens (the
+last three on the MMA product); int32 and BitLinear outputs.
 """
 import json
 import os
@@ -28,14 +28,14 @@ out = {}
 SHAPES = [(1, 512), (5, 640), (31, 700), (33, 1000), (100, 3200), (257, 2560), (1000, 5120), (70, 10240),
           (65, 16384), (300, 27648), (4800, 3200)]
 for (N, K) in SHAPES:
-    for M in (1, 3, 8):
+    for M in (1, 3, 8, 13):
         q, w = synth.uniform_int8_ternary(N, K, seed=N + K + M, M=M)
         q[0, :5] = -128
         packed = bn.bitnet_pack_weights(torch.from_numpy(w).cuda())
         y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), packed, N).cpu().numpy()
         ok_i = bool(np.array_equal(y, oracle.gemm_i32(q, w)))
         ok_b = True
-        if M in (1, 3):
+        if M in (1, 3, 13):
             x, W = synth.bitlinear_inputs(M, N, K, seed=N + M)
             g = oracle.absmean(W)
             wt = oracle.ternarize(W, g)
@@ -53,9 +53,10 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores":
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma":
 # variant 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp), rows
-# per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM)
+# per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM), mma =
+# 1 / 0 the MMA or the dp4a product for one token
 @pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
                                   "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
                                   "0,0,0,0,-1,0,3",      # 16 warps, ring up to 2
@@ -65,7 +66,11 @@ print(json.dumps(out))
                                   "0,0,0,0,-1,0,-1,0,-1,0,16",   # 16-row blocks (two lanes per row)
                                   "0,0,0,0,-1,0,1,0,-1,0,16",    # 16-row blocks, 8 warps, ring up to 4
                                   "0,0,0,0,-1,0,-1,0,-1,0,0,1",  # co-residency mode (16-row blocks below 148)
-                                  "0,0,0,0,-1,0,-1,0,-1,0,32,1"])  # co-residency mode, 32-row blocks
+                                  "0,0,0,0,-1,0,-1,0,-1,0,32,1",  # co-residency mode, 32-row blocks
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,1",  # MMA product for one token too
+                                  "0,0,0,0,-1,0,1,0,-1,0,16,-1,1",  # MMA, 16-row blocks, 8 warps
+                                  "0,0,0,0,-1,0,2,0,-1,0,0,-1,1",  # MMA, 12 warps
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,0"])  # dp4a product for one token
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
