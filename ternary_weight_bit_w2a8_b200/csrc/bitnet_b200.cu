@@ -302,22 +302,28 @@ constexpr int kTmaNumCfg = 5;
 constexpr int kTmaCfg[kTmaNumCfg][2] = {{8, 4}, {12, 3}, {16, 2}, {8, 2}, {4, 4}};
 using TmaKernel = void (*)(const CUtensorMap, const GemvTmaArgs);
 
-// BitLinear with up to this many tokens quantises them inside the GEMV's
-// prologue (every CTA reads and quantises all of them); more tokens are
-// quantised once by quant_act_kernel first.  Measured on B200, 2560 x 6912:
-// 2 tokens 6.2 us fused vs 7.8 us in two passes; 8 tokens 17.4 vs 15.4 us.
-constexpr int kFusedQuantMaxTokens = 4;
-
 // Tokens per TMA GEMV launch: up to this many tokens read the weights once in
 // one GEMV launch (on the MMA path from 2 tokens up); more go to the
 // tensor-core GEMM.
 constexpr int kGemvMaxTokens = 16;
 
+// BitLinear with up to this many tokens quantises them inside the GEMV's
+// prologue (every CTA reads and quantises all of them); more tokens are
+// quantised once by quant_act_kernel first.  The tuning field `fuse` moves
+// the boundary: 1 quantises every token count inside the launch, 0 every
+// count above one in a pass of its own.
+constexpr int kFusedQuantMaxTokens = 4;
+
+int fused_quant_max_tokens() {
+    const int f = gemv_tune().fuse;
+    return f == 1 ? kGemvMaxTokens : (f == 0 ? 1 : kFusedQuantMaxTokens);
+}
+
 // Kernel of (mode, warps, tokens per launch, rows per block, MMA): one token
 // on 4, 8, 12 or 16 warps with dp4a or the MMA path, several tokens (MT = 2,
 // 4, 8, 16) on 8 or 16 warps with the MMA path, for int8 activations (xmode 0)
-// and, up to kFusedQuantMaxTokens tokens, bf16 activations quantised in the
-// kernel (xmode 1); row blocks of 32 or 16 rows.  Slot in the shared-memory
+// or bf16 activations quantised in the kernel (xmode 1); row blocks of 32 or
+// 16 rows.  Slot in the shared-memory
 // opt-in table, -1 if no such kernel.
 constexpr int kTmaNumSlots = 2 * 2 * 2 * kTmaNumCfg * 5;
 static_assert(kTmaNumSlots <= (int)(sizeof(DeviceInfo::tma_max_dyn) / sizeof(size_t)), "opt-in table");
@@ -326,7 +332,6 @@ int tma_kernel_slot(int xmode, int cfg, int mt, int rows, int mma) {
     const int W = kTmaCfg[cfg][0];
     const int mti = mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : (mt == 8 ? 3 : (mt == 16 ? 4 : -1))));
     if (mti < 0 || (mt > 1 && (!mma || (W != 8 && W != 16)))) return -1;
-    if (xmode == 1 && mt > kFusedQuantMaxTokens) return -1;
     return (((xmode * 2 + (rows == 16 ? 1 : 0)) * 2 + (mma ? 1 : 0)) * kTmaNumCfg + cfg) * 5 + mti;
 }
 
@@ -345,11 +350,9 @@ TmaKernel tma_kernel_w(int W, int mt) {
         switch (mt) {
             case 2: return w16 ? gemv_tma_kernel<X, 16, 2, R, 1> : gemv_tma_kernel<X, 8, 2, R, 1>;
             case 4: return w16 ? gemv_tma_kernel<X, 16, 4, R, 1> : gemv_tma_kernel<X, 8, 4, R, 1>;
+            case 8: return w16 ? gemv_tma_kernel<X, 16, 8, R, 1> : gemv_tma_kernel<X, 8, 8, R, 1>;
+            case 16: return w16 ? gemv_tma_kernel<X, 16, 16, R, 1> : gemv_tma_kernel<X, 8, 16, R, 1>;
             default: break;
-        }
-        if constexpr (X == 0) {
-            if (mt == 8) return w16 ? gemv_tma_kernel<0, 16, 8, R, 1> : gemv_tma_kernel<0, 8, 8, R, 1>;
-            if (mt == 16) return w16 ? gemv_tma_kernel<0, 16, 16, R, 1> : gemv_tma_kernel<0, 8, 16, R, 1>;
         }
     }
     return nullptr;
@@ -829,7 +832,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool q_tma_ok, bool bitlinea
             p.ws_bytes = tp.ws_bytes;
             // BitLinear on more tokens than the fused prologue takes quantises
             // them once into the workspace (before the GEMV's own scratch)
-            if (bitlinear && M > kFusedQuantMaxTokens) p.ws_bytes += round_up(M * K, 256) + round_up(M * 4, 256);
+            if (bitlinear && M > fused_quant_max_tokens())
+                p.ws_bytes += round_up(M * K, 256) + round_up(M * 4, 256);
             return p;
         }
     }
@@ -1016,7 +1020,7 @@ BITNET_API int bitnet_bitlinear(const uint16_t *x, const uint8_t *packed, const 
         fill_kernel<uint16_t><<<grid_for(M * N, kThreads * 4, dev->sm_count), kThreads, 0, st>>>(y, M * N, 0);
         return launched();
     }
-    if (p.path == kPathGemv && M > kFusedQuantMaxTokens && M <= kGemvMaxTokens && tma_plan(M, N, K).use) {
+    if (p.path == kPathGemv && M > fused_quant_max_tokens() && M <= kGemvMaxTokens && tma_plan(M, N, K).use) {
         // small batch: quantise the tokens once, then one pass over the weights
         int8_t *q = static_cast<int8_t *>(workspace);
         float *s = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(M * K, 256));

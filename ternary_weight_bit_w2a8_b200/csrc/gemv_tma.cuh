@@ -353,6 +353,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ float red[(XMODE == 1 ? MT : 1) * 32];
+    __shared__ float fsh[MT];  // BitLinear rescale factors gamma / s_t
     // the descriptor fetch is the first long latency of the launch: start it now
     if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     const int ns = a.ns, slices = a.slices;
@@ -418,21 +419,20 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     pdl_launch_dependents();
     pdl_wait();
 
-    float sc[MT];
-    if (XMODE == 0) {
-        stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq);
+    {
+        float sc[MT];
+        if (XMODE == 0) {
+            stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq);
+        } else {
+            stage_tokens_bf16<MT>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
+        }
+        if (threadIdx.x == 0) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) sc[t] = 0.0f;
-    } else {
-        stage_tokens_bf16<MT>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
+            for (int t = 0; t < MT; ++t)
+                fsh[t] = (t < a.M && a.y_bf16 != nullptr) ? __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]) : 0.0f;
+        }
     }
     __syncthreads();
-    float f[MT];
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-        f[t] = 0.0f;
-        if (t < a.M && a.y_bf16 != nullptr) f[t] = __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]);
-    }
 
     // dp4a accumulators: one row (or half of one), per code plane
     int acc[4] = {0, 0, 0, 0}, corr = 0;
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
                 const int tot = atomicAdd(&accs[(sl * MT + t) * ROWS + brow], 0);
                 if (part == 0 && t < a.M && n < a.N) {
                     if (a.y_bf16 != nullptr)
-                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, f[t]));
+                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, fsh[t]));
                     else
                         a.y_i32[(int64_t)t * a.N + n] = tot;
                 }
