@@ -405,7 +405,9 @@ def measure_small_batch(torch, bn, shapes, ms_list, warmup, l2_bytes, reps=30):
             y = torch.empty((M, N), dtype=torch.int32, device="cuda")
             yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
             ws = bn.workspace(M, N, K)
-            row = {"M": M, "N": N, "K": K}
+            # the library's plan: one weight pass of the TMA GEMV (m16n8k32 MMA
+            # product) up to 16 tokens, the tcgen05 GEMM beyond
+            row = {"M": M, "N": N, "K": K, "path": "gemv_tma_mma" if M <= 16 else "gemm_tcgen05"}
             for name, fn in (("int32", lambda i: bn.bitnet_w2a8_gemm(q, copies[i % C], N, y=y, ws=ws)),
                              ("bitlinear", lambda i: bn.bitnet_bitlinear(x, copies[i % C], gamma, N, y=yb, ws=ws))):
                 def run(fn=fn):
@@ -541,7 +543,7 @@ def run_ours(args, rank, world, dist):
         torch.cuda.empty_cache()
         details["bitlinear_decode"] = measure_bitlinear_decode(torch, bn, synth.BITLINEAR_DECODE_SHAPES,
                                                                args.warmup, l2)
-        details["small_batch"] = measure_small_batch(torch, bn, synth.BITLINEAR_DECODE_SHAPES, [2, 4, 8, 16, 32, 64],
+        details["small_batch"] = measure_small_batch(torch, bn, synth.BITLINEAR_DECODE_SHAPES, [2, 4, 8, 12, 16, 32, 64],
                                                      args.warmup, l2)
         details["prefill"] = measure_prefill(torch, bn, synth.PREFILL_M, synth.PREFILL_SHAPES, args.warmup, int8_peak)
         bf = measure_bf16_context(torch, synth.SWEEP_SHAPES, args.warmup, l2)

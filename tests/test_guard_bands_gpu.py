@@ -50,6 +50,8 @@ def bf16_ok(y, y_ref):
 GEMM_CASES = [
     (1, 257, 2560),    # TMA GEMV, ragged last row block
     (1, 1000, 5120),   # TMA GEMV, several row blocks per CTA
+    (1, 5115, 27648),  # TMA GEMV, 160 row blocks on 148 CTAs (12 take two), ragged last block
+    (13, 300, 2560),   # small batch, 16-token MMA tiles
     (1, 300, 300),     # register GEMV (K < 512)
     (1, 64, 65536),    # register GEMV... or TMA; either way the plan's scratch is guarded
     (1, 20, 200000),   # K-split register GEMV: int32 partials in the workspace

@@ -21,31 +21,37 @@ CHILD = r"""
 import json, sys
 import numpy as np, torch
 sys.path.insert(0, ROOT)
+sys.path.insert(0, ROOT + "/tests")
 import oracle
+from guarded import Guarded
 import ternary_weight_bit_w2a8_b200 as bn
 from ternary_weight_bit_w2a8_b200 import synth
 out = {}
 SHAPES = [(1, 512), (5, 640), (31, 700), (33, 1000), (100, 3200), (257, 2560), (1000, 5120), (70, 10240),
-          (65, 16384), (300, 27648), (4800, 3200)]
+          (65, 16384), (300, 27648), (4800, 3200), (4832, 27648), (20000, 3200)]
 for (N, K) in SHAPES:
     for M in (1, 3, 8, 13):
         q, w = synth.uniform_int8_ternary(N, K, seed=N + K + M, M=M)
         q[0, :5] = -128
         packed = bn.bitnet_pack_weights(torch.from_numpy(w).cuda())
-        y = bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), packed, N).cpu().numpy()
-        ok_i = bool(np.array_equal(y, oracle.gemm_i32(q, w)))
+        yg = Guarded(torch, (M, N), torch.int32, fill=-7)
+        bn.bitnet_w2a8_gemm(torch.from_numpy(q).cuda(), packed, N, y=yg.t)
+        ok_i = bool(np.array_equal(yg.t.cpu().numpy(), oracle.gemm_i32(q, w))) and yg.intact()
         ok_b = True
         if M in (1, 3, 13):
             x, W = synth.bitlinear_inputs(M, N, K, seed=N + M)
             g = oracle.absmean(W)
             wt = oracle.ternarize(W, g)
-            yb = bn.bitnet_bitlinear(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16),
-                                     bn.bitnet_pack_weights(torch.from_numpy(wt).cuda()),
-                                     torch.tensor([float(g)], dtype=torch.float32, device="cuda"), N)
+            ybg = Guarded(torch, (M, N), torch.int16, fill=0x7F7F)
+            bn.bitnet_bitlinear(torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16),
+                                bn.bitnet_pack_weights(torch.from_numpy(wt).cuda()),
+                                torch.tensor([float(g)], dtype=torch.float32, device="cuda"), N,
+                                y=ybg.t.view(torch.bfloat16))
+            yb = ybg.t.view(torch.bfloat16)
             yr = oracle.bitlinear(x, wt, g)[0]
             yf = yb.float().cpu().numpy().astype(np.float64)
             err = np.abs(yf - yr)
-            ok_b = bool(np.where(np.abs(yr) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(yr)).all())
+            ok_b = bool(np.where(np.abs(yr) < 0.1, err <= 1e-3, err <= 1e-2 * np.abs(yr)).all()) and ybg.intact()
         out[f"{M}x{N}x{K}"] = [ok_i, ok_b]
 torch.cuda.synchronize()
 out["device_error"] = bn.bitnet_get_device_error()
@@ -53,10 +59,12 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma":
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma,split,w0":
 # variant 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp), rows
 # per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM), mma =
-# 1 / 0 the MMA or the dp4a product for one token
+# 1 / 0 the MMA or the dp4a product for one token, split = 1 / 0 always /
+# never deal leftover row blocks' items over all CTAs (4832 x 27648 and 20000 x
+# 3200 have 3 and 136 leftover 32-row blocks), w0 = items fewer for warp 0
 @pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
                                   "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
                                   "0,0,0,0,-1,0,3",      # 16 warps, ring up to 2
@@ -70,7 +78,11 @@ print(json.dumps(out))
                                   "0,0,0,0,-1,0,-1,0,-1,0,0,-1,1",  # MMA product for one token too
                                   "0,0,0,0,-1,0,1,0,-1,0,16,-1,1",  # MMA, 16-row blocks, 8 warps
                                   "0,0,0,0,-1,0,2,0,-1,0,0,-1,1",  # MMA, 12 warps
-                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,0"])  # dp4a product for one token
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,0",  # dp4a product for one token
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,1,0",  # split wherever possible
+                                  "0,0,0,0,-1,0,-1,0,-1,0,16,-1,-1,1,3",  # split, 16-row blocks, warp 0 lighter
+                                  "0,0,0,0,-1,0,1,0,-1,0,0,-1,1,1,2",  # split, MMA product, 8 warps
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,0"])  # never split
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
