@@ -120,18 +120,17 @@ struct GemvSplit {
 };
 
 // optional override:
-// BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores,mma,split,w0"
+// BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores,mma,l2"
 // (register GEMV: G, R, U, ctas, prefetch, S; TMA GEMV: tma = 0 off or
 // 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth, rows per block 16 or
 // 32, cores = 1 the co-residency mode (see tma_plan), mma = 1 / 0 the MMA or
-// dp4a product for one token, split = 0 / 1 never / always deal the remainder
-// row blocks' items over all CTAs, w0 = items fewer for warp 0 then;
-// tensor-core GEMM: R < 0
+// dp4a product for one token, l2 = 0 weights read without the L2
+// evict-first policy; tensor-core GEMM: R < 0
 // variant, S K-splits, fuse = 1 quantises BitLinear activations inside the
 // GEMM launch; activation quantisation: qwpt warps per token, 1..8)
 struct GemvTune {
     int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1, qwpt = 0, rows = 0,
-        cores = -1, mma = -1, split = -1, w0 = -1;
+        cores = -1, mma = -1, l2 = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -140,8 +139,8 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S,
-                   &t.tma, &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores, &t.mma, &t.split, &t.w0);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S,
+                   &t.tma, &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores, &t.mma, &t.l2);
     });
     return t;
 }
@@ -416,9 +415,6 @@ struct TmaPlan {
     int mt;            // tokens per launch (1, 2, 4, 8, 16)
     int rows;          // rows per block (32 or 16)
     int mma;           // 1: the MMA product, 0: dp4a (one token only)
-    int64_t whole;     // split mode: whole row blocks per CTA
-    int64_t split_items;  // split mode: items of the remainder blocks (0: no split)
-    int w0_lighter;    // split mode: items fewer for warp 0
     int64_t nblocks;
     size_t smem;
     int64_t ws_bytes;  // always 0: the TMA GEMV needs no workspace
@@ -457,34 +453,7 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     const int64_t gmax = (int64_t)kRefSMs * per_sm;
     p.grid = (int)(p.nblocks < gmax ? p.nblocks : gmax);
     p.max_blocks = (int)ceil_div(p.nblocks, p.grid);
-    int64_t max_items = (int64_t)p.max_blocks * p.slices;
-    // split mode (tuning field split = 1): with whole = floor(blocks / grid)
-    // >= 1 and R blocks left over, every CTA takes `whole` blocks and an even
-    // share of the R blocks' items instead of R CTAs taking one block more
-    // (5120 x 27648 on 148 SMs: 59 instead of 108 boxes for the busiest CTA).
-    // Measured on B200 it is slower wherever it applies (5120 x 27648: 12.6
-    // vs 11.7 us; 20480 x 3200: 8.3 vs 6.1 us): with every SM streaming, a
-    // CTA's share of the weights comes no faster than the busiest CTA's whole
-    // blocks do alone, and the cross-CTA sum adds a chain of global-memory
-    // round trips at the end.  Not the default.
-    if (p.mt == 1 && tn.split == 1 && p.nblocks > p.grid) {
-        const int64_t G = p.grid, whole = p.nblocks / G, R = p.nblocks - whole * G, RS = R * p.slices;
-        if (R > 0 && R <= kSplitMaxBlocks && RS >= G) {
-            const int64_t spl = whole * p.slices + ceil_div(RS, G);
-            p.whole = whole;
-            p.split_items = RS;
-            p.w0_lighter = tn.w0 >= 0 ? tn.w0 : 1;
-            int most = 0;  // split slots of the CTA that touches the most split blocks
-            for (int64_t c = 0; c < G; ++c) {
-                const int64_t a0 = c * RS / G, a1 = (c + 1) * RS / G;
-                const int n = a1 > a0 ? (int)((a1 - 1) / p.slices - a0 / p.slices + 1) : 0;
-                if (n > most) most = n;
-            }
-            p.max_blocks = (int)whole + most;
-            max_items = spl;
-        }
-    }
-    const int64_t ipw = ceil_div(max_items + p.w0_lighter, W);
+    const int64_t ipw = ceil_div((int64_t)p.max_blocks * p.slices, W);
     p.ns = (int)(ipw < NS ? (ipw < 1 ? 1 : ipw) : NS);
     if (tn.ns > 0) p.ns = tn.ns < NS ? tn.ns : NS;
     auto bytes = [&](int ns) { return gemv_tma_smem_bytes(W, ns, p.slices, p.max_blocks, p.mt, p.rows); };
@@ -537,13 +506,7 @@ int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t 
     a.gamma = gamma;
     a.s_act = s_act;
     a.test_stall = test_stall;
-    a.whole = tp.whole;
-    a.split_items = tp.split_items;
-    a.w0_lighter = tp.w0_lighter;
-    if (tp.split_items > 0) {
-        static std::atomic<uint32_t> slot{0};
-        a.split_slot = (int)(slot.fetch_add(1, std::memory_order_relaxed) % kSplitSlots);
-    }
+    a.evict_first = gemv_tune().l2 == 0 ? 0 : 1;  // measured on B200: 25.9 -> 25.6 us per sweep step
     return launched(launch_pdl(kern, dim3(tp.grid), dim3(kTmaCfg[tp.cfg][0] * 32), tp.smem, st, map, a));
 }
 
@@ -1124,16 +1087,9 @@ BITNET_API int bitnet_get_device_error(void *stream) {
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BITNET_ERR_CUDA;
-        // a launch that gave up may have left a grid barrier half-counted, or
-        // a split row block's sums and counter behind
+        // a launch that gave up may have left a grid barrier half-counted
         static const unsigned int zeros[kGridBarSlots] = {};
         if (cudaMemcpyToSymbol(g_grid_bar, zeros, sizeof(zeros)) != cudaSuccess) return BITNET_ERR_CUDA;
-        void *acc = nullptr, *cnt = nullptr;
-        if (cudaGetSymbolAddress(&acc, g_split_acc) != cudaSuccess ||
-            cudaGetSymbolAddress(&cnt, g_split_cnt) != cudaSuccess ||
-            cudaMemset(acc, 0, sizeof(g_split_acc)) != cudaSuccess ||
-            cudaMemset(cnt, 0, sizeof(g_split_cnt)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
-            return BITNET_ERR_CUDA;
     }
     return v;
 }

@@ -65,24 +65,8 @@ struct GemvTmaArgs {
     const float *gamma;   // weight scale (BitLinear)
     const float *s_act;   // mode 0 with bf16 output: per-token activation scales [M]
     int test_stall;       // test hook: warp 0 never requests its first box, so its first wait times out
-    // split mode (one token; split_items > 0): CTA c owns the whole row
-    // blocks c + k * gridDim.x, k < whole, and a contiguous range of the
-    // split_items (row block, slice) items of the last nblocks - whole *
-    // gridDim.x blocks, [c * split_items / G, (c + 1) * split_items / G);
-    // those blocks' partial sums meet in g_split_acc[split_slot]
-    int64_t whole;
-    int64_t split_items;
-    int split_slot;
-    int w0_lighter;       // split mode: items fewer for warp 0, which takes the CTA's split items first
+    int evict_first;      // 1: weight boxes are read with the L2 evict-first policy
 };
-
-// Cross-CTA sums of split row blocks, one slot per launch (a ring the host
-// deals out), zero at rest: the last contributor of a block reads the total,
-// writes the outputs and zeroes the block's words and counter again.
-constexpr int kSplitSlots = 64;
-constexpr int kSplitMaxBlocks = 256;
-__device__ int g_split_acc[kSplitSlots][kSplitMaxBlocks * 32];
-__device__ unsigned int g_split_cnt[kSplitSlots][kSplitMaxBlocks];
 
 // Dynamic shared memory of a launch: ring of warps x stages boxes of `rows`
 // rows, linear activations, per-row-block accumulators and counters, slice
@@ -150,6 +134,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
             if (mbar_try_wait(bar, parity)) return true;
         if (global_timer_ns() - t0 > kWaitLimitNs) return false;
     }
+}
+
+// L2 policy for data read once per call (the packed weights): its lines are
+// the first to go, so that what the next calls reuse stays in L2 (kernel
+// code, activations, outputs, tensor maps).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void tma_load_box_hint(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                                  uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+        "%3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
 }
 
 __device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
@@ -392,63 +394,31 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int brow = lane / kLPR, part = lane % kLPR;  // this lane's box row and chunk half
     const int mg = lane >> 2, mt4 = lane & 3;          // MMA fragment coordinates (g, t)
-    // this CTA's items: its split items (split mode), then its whole row
-    // blocks, each in (row block, slice) order; one accumulator slot per row
-    // block touched, the split blocks' first
-    const bool split = MT == 1 && a.split_items > 0;
-    const int64_t s0 = split ? cid * a.split_items / ncl : 0, s1 = split ? (cid + 1) * a.split_items / ncl : 0;
-    const int n_split = (int)(s1 - s0);
-    const int sb0 = (int)(s0 / slices);                                        // first split block (of the split ones)
-    const int n_sslots = n_split > 0 ? (int)((s1 - 1) / slices) - sb0 + 1 : 0;
-    const int64_t nb_whole = split ? a.whole : (a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0);
-    const int64_t items = n_split + nb_whole * slices;
-    const int nslots = n_sslots + (int)nb_whole;
-    auto blk_of = [&](int sl) -> int64_t {  // row block of a slot
-        return a.blk_begin + (sl < n_sslots ? a.whole * ncl + sb0 + sl : cid + (int64_t)(sl - n_sslots) * ncl);
-    };
-    auto expected = [&](int sl) -> int {  // the CTA's items in a slot
-        if (sl >= n_sslots) return slices;
-        const int64_t b0 = (int64_t)(sb0 + sl) * slices;
-        return (int)(min(s1, b0 + slices) - max(s0, b0));
-    };
-    // this warp's items: a contiguous range of the CTA's items (warp 0's
-    // shorter by w0_lighter in split mode: it meets the other CTAs first)
-    const int64_t lighter = n_split > 0 ? a.w0_lighter : 0;
-    const int64_t ipw = ceil_div(items + lighter, W);
-    const int64_t it_begin = min(items, max((int64_t)0, warp * ipw - lighter));
-    const int n_items = (int)max((int64_t)0, min(items, (warp + 1) * ipw - lighter) - it_begin);
+    // this CTA's items, in (row block, slice) order
+    const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
+    const int64_t items = nb_cta * slices;
+    const int nslots = (int)nb_cta;
+    // this warp's items: a contiguous range of the CTA's items
+    const int64_t ipw = ceil_div(items, W);
+    const int64_t it_begin = min(items, warp * ipw);
+    const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
     uint64_t *mybar = bars + warp * ns;
     uint8_t *myring = ring + warp * ns * kBoxBytes;
-    // (slot, slice) of CTA item i, and the step to item i + 1
-    auto locate = [&](int64_t i, int &sl, int &j) {
-        if (i < n_split) {
-            const int64_t g = s0 + i;
-            sl = (int)(g / slices) - sb0;
-            j = (int)(g % slices);
-        } else {
-            sl = n_sslots + (int)((i - n_split) / slices);
-            j = (int)((i - n_split) % slices);
-        }
-    };
-    auto step = [&](int64_t &i, int &sl, int &j) {  // true when the step leaves slot sl
-        ++i;
-        if (++j == slices || i == n_split) {
-            j = 0;
-            ++sl;
-            return true;
-        }
-        return false;
-    };
 
-    // producer cursor over the warp's items
-    int64_t iitem = it_begin;
-    int islot, ij;
-    locate(it_begin, islot, ij);
+    // cursor over the warp's items: (slot, slice); row block = cid + slot * ncl
+    int islot = (int)(it_begin / slices), ij = (int)(it_begin - (int64_t)islot * slices);
+    const uint64_t wpolicy = l2_evict_first_policy();
     auto issue_next = [&](int s) {
-        const int64_t row0 = blk_of(islot) * ROWS;
+        const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * ROWS;
         mbar_arrive_expect_tx(&mybar[s], kBoxBytes);
-        tma_load_box(myring + s * kBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
-        step(iitem, islot, ij);
+        if (a.evict_first)
+            tma_load_box_hint(myring + s * kBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s], wpolicy);
+        else
+            tma_load_box(myring + s * kBoxBytes, &wmap, ij * kTmaSliceBytes, (int)row0, &mybar[s]);
+        if (++ij == slices) {
+            ij = 0;
+            ++islot;
+        }
     };
     // weights do not depend on the previous kernel: request them before waiting
     // for it.  A warp's ring and barriers are its own, so lane 0 sets them up
@@ -458,7 +428,10 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int s = 0; s < ns && s < n_items; ++s) {
             if (s == 0 && warp == 0 && a.test_stall) {  // skip the request: nothing completes this stage
-                step(iitem, islot, ij);
+                if (++ij == slices) {
+                    ij = 0;
+                    ++islot;
+                }
                 continue;
             }
             issue_next(s);
@@ -505,44 +478,6 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     };
     zero_acc();
     int ncontrib = 0;
-    // split block of slot sl (one token): adds this CTA's sums into the
-    // launch's global accumulator; the last of the block's CTAs reads the
-    // total, writes the outputs and zeroes the accumulator and counter
-    auto combine = [&](int sl) {
-        const int r = sb0 + sl;
-        int *gacc = &g_split_acc[a.split_slot][r * ROWS];
-        unsigned int *gcnt = &g_split_cnt[a.split_slot][r];
-        const int mine = atomicAdd(&accs[sl * ROWS + brow], 0);
-        if (part == 0) atomicAdd(&gacc[brow], mine);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            // CTAs whose item ranges meet block r (every range is non-empty)
-            const int64_t G = ncl, RS = a.split_items;
-            const int64_t g0 = (int64_t)r * slices, g1 = g0 + slices - 1;
-            const int64_t c0 = ((g0 + 1) * G - 1) / RS, c1 = ((g1 + 1) * G - 1) / RS;
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            last = (atomicAdd(gcnt, 1u) + 1u == (unsigned int)(c1 - c0 + 1));
-            if (last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            const int64_t n = blk_of(sl) * ROWS + brow;
-            if (part == 0) {
-                const int tot = __ldcg(&gacc[brow]);
-                if (n < a.N) {
-                    if (a.y_bf16 != nullptr)
-                        a.y_bf16[n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, fsh[0]));
-                    else
-                        a.y_i32[n] = tot;
-                }
-                gacc[brow] = 0;
-            }
-            if (lane == 0) *gcnt = 0u;
-        }
-    };
-    constexpr int kMaxPend = 4;
-    int pend[kMaxPend], npend = 0;
     // folds this warp's partial sums of slot `sl` into shared memory (the
     // activation-sum correction is taken once per row and token); the warp
     // completing the slot's items writes its results
@@ -572,18 +507,11 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
         __threadfence_block();
         __syncwarp();
         int fin = 0;
-        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == expected(sl));
+        if (lane == 0) fin = (atomicAdd(&done[sl], ncontrib) + ncontrib == slices);
         fin = __shfl_sync(0xffffffffu, fin, 0);
-        if (fin && MT == 1 && sl < n_sslots) {
-            // a split block: its cross-CTA sum is taken after this warp's last
-            // item, off the path of the weight stream
-            if (npend < kMaxPend)
-                pend[npend++] = sl;
-            else
-                combine(sl);
-        } else if (fin) {
+        if (fin) {
             __threadfence_block();
-            const int64_t n = blk_of(sl) * ROWS + brow;
+            const int64_t n = (a.blk_begin + cid + (int64_t)sl * ncl) * ROWS + brow;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
                 const int tot = atomicAdd(&accs[(sl * MT + t) * ROWS + brow], 0);
@@ -599,10 +527,8 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
         ncontrib = 0;
     };
 
-    // consumer cursor
-    int64_t citem = it_begin;
-    int cslot, cj;
-    locate(it_begin, cslot, cj);
+    // consume cursor
+    int cslot = (int)(it_begin / slices), cj = (int)(it_begin - (int64_t)cslot * slices);
     int s = 0;
     uint32_t phase = 0;
     for (int n = 0; n < n_items; ++n) {
@@ -679,10 +605,12 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
             s = 0;
             phase ^= 1u;
         }
-        const int sl = cslot;
-        if (step(citem, cslot, cj) || n + 1 == n_items) flush(sl);
+        if (++cj == slices || n + 1 == n_items) {
+            flush(cslot);
+            cj = 0;
+            ++cslot;
+        }
     }
-    for (int i = 0; i < npend; ++i) combine(pend[i]);
 }
 
 }  // namespace bitnet

@@ -59,12 +59,12 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma,split,w0":
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma,l2":
 # variant 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp), rows
 # per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM), mma =
-# 1 / 0 the MMA or the dp4a product for one token, split = 1 / 0 always /
-# never deal leftover row blocks' items over all CTAs (4832 x 27648 and 20000 x
-# 3200 have 3 and 136 leftover 32-row blocks), w0 = items fewer for warp 0
+# 1 / 0 the MMA or the dp4a product for one token, l2 = 0 weights without the
+# L2 evict-first policy.  4832 x 27648 and 20000 x
+# 3200 leave 3 and 136 CTAs with one 32-row block more than the others.
 @pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
                                   "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
                                   "0,0,0,0,-1,0,3",      # 16 warps, ring up to 2
@@ -79,10 +79,7 @@ print(json.dumps(out))
                                   "0,0,0,0,-1,0,1,0,-1,0,16,-1,1",  # MMA, 16-row blocks, 8 warps
                                   "0,0,0,0,-1,0,2,0,-1,0,0,-1,1",  # MMA, 12 warps
                                   "0,0,0,0,-1,0,-1,0,-1,0,0,-1,0",  # dp4a product for one token
-                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,1,0",  # split wherever possible
-                                  "0,0,0,0,-1,0,-1,0,-1,0,16,-1,-1,1,3",  # split, 16-row blocks, warp 0 lighter
-                                  "0,0,0,0,-1,0,1,0,-1,0,0,-1,1,1,2",  # split, MMA product, 8 warps
-                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,0"])  # never split
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,0"])  # weights without the evict-first policy
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
