@@ -376,7 +376,9 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     // the descriptor fetch is the first long latency of the launch: start it now
     if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     const int ns = a.ns, slices = a.slices;
-    const int64_t cid = blockIdx.x, ncl = gridDim.x;  // row blocks cid, cid + ncl, ...
+    // row blocks cid, cid + ncl, ...; index arithmetic in 32 bits: the
+    // divisions on the way to the first weight request stay short
+    const int cid = blockIdx.x, ncl = gridDim.x;
     const int64_t kq = (int64_t)slices * kTmaSliceK;
     const int64_t ldx = gemv_tma_token_stride(slices, MT);
 
@@ -395,18 +397,20 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     const int brow = lane / kLPR, part = lane % kLPR;  // this lane's box row and chunk half
     const int mg = lane >> 2, mt4 = lane & 3;          // MMA fragment coordinates (g, t)
     // this CTA's items, in (row block, slice) order
-    const int64_t nb_cta = a.nblocks > cid ? ceil_div(a.nblocks - cid, ncl) : 0;
-    const int64_t items = nb_cta * slices;
-    const int nslots = (int)nb_cta;
+    const int nblk = (int)a.nblocks;
+    const int nb_cta = nblk > cid ? (nblk - cid + ncl - 1) / ncl : 0;
+    const int items = nb_cta * slices;
+    const int nslots = nb_cta;
     // this warp's items: a contiguous range of the CTA's items
-    const int64_t ipw = ceil_div(items, W);
-    const int64_t it_begin = min(items, warp * ipw);
-    const int n_items = (int)(min(items, it_begin + ipw) - it_begin);
+    const int ipw = (items + W - 1) / W;
+    const int it_begin = min(items, warp * ipw);
+    const int n_items = min(items, it_begin + ipw) - it_begin;
     uint64_t *mybar = bars + warp * ns;
     uint8_t *myring = ring + warp * ns * kBoxBytes;
 
     // cursor over the warp's items: (slot, slice); row block = cid + slot * ncl
-    int islot = (int)(it_begin / slices), ij = (int)(it_begin - (int64_t)islot * slices);
+    int islot = it_begin / slices, ij = it_begin - islot * slices;
+    const int cslot0 = islot, cj0 = ij;  // the consumer starts where the producer does
     const uint64_t wpolicy = l2_evict_first_policy();
     auto issue_next = [&](int s) {
         const int64_t row0 = (a.blk_begin + cid + (int64_t)islot * ncl) * ROWS;
@@ -528,7 +532,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     };
 
     // consume cursor
-    int cslot = (int)(it_begin / slices), cj = (int)(it_begin - (int64_t)cslot * slices);
+    int cslot = cslot0, cj = cj0;
     int s = 0;
     uint32_t phase = 0;
     for (int n = 0; n < n_items; ++n) {
