@@ -37,7 +37,7 @@ struct DeviceInfo {
     int status = BITNET_OK;
     int sm_count = 0;
     uint64_t smem_attr_set = 0;  // GEMV instantiations whose shared-memory limit is raised
-    size_t tma_max_dyn[200] = {};  // dynamic shared memory opted into by each TMA GEMV variant
+    size_t tma_max_dyn[400] = {};  // dynamic shared memory opted into by each TMA GEMV variant
     bool tc_attr_set[2 * 10] = {};    // shared-memory opt-in done, per tensor-core GEMM variant
     size_t smem_optin = 0;       // largest dynamic shared memory a CTA may opt into
     int n_occ = 0;
@@ -120,17 +120,18 @@ struct GemvSplit {
 };
 
 // optional override:
-// BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores,mma,l2"
+// BITNET_GEMV_TUNE="G,R,U,ctas_per_sm,prefetch_tasks,S,tma,ns,fuse,qwpt,rows,cores,mma,l2,sflags"
 // (register GEMV: G, R, U, ctas, prefetch, S; TMA GEMV: tma = 0 off or
 // 1..5 a variant of kTmaCfg, ctas per SM, ns ring depth, rows per block 16 or
 // 32, cores = 1 the co-residency mode (see tma_plan), mma = 1 / 0 the MMA or
 // dp4a product for one token, l2 = 0 weights read without the L2
-// evict-first policy; tensor-core GEMM: R < 0
+// evict-first policy, sflags = 1 / 0 per-slice staging barriers always /
+// never; tensor-core GEMM: R < 0
 // variant, S K-splits, fuse = 1 quantises BitLinear activations inside the
 // GEMM launch; activation quantisation: qwpt warps per token, 1..8)
 struct GemvTune {
     int G = 0, R = 0, U = 0, ctas = 0, prefetch = -1, S = 0, tma = -1, ns = 0, fuse = -1, qwpt = 0, rows = 0,
-        cores = -1, mma = -1, l2 = -1;
+        cores = -1, mma = -1, l2 = -1, sflags = -1;
 };
 
 const GemvTune &gemv_tune() {
@@ -139,8 +140,8 @@ const GemvTune &gemv_tune() {
     std::call_once(once, [] {
         const char *e = getenv("BITNET_GEMV_TUNE");
         if (e != nullptr)
-            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S,
-                   &t.tma, &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores, &t.mma, &t.l2);
+            sscanf(e, "%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d,%d", &t.G, &t.R, &t.U, &t.ctas, &t.prefetch, &t.S,
+                   &t.tma, &t.ns, &t.fuse, &t.qwpt, &t.rows, &t.cores, &t.mma, &t.l2, &t.sflags);
     });
     return t;
 }
@@ -327,14 +328,15 @@ int fused_quant_max_tokens() {
 // or bf16 activations quantised in the kernel (xmode 1); row blocks of 32 or
 // 16 rows.  Slot in the shared-memory
 // opt-in table, -1 if no such kernel.
-constexpr int kTmaNumSlots = 2 * 2 * 2 * kTmaNumCfg * 5;
+constexpr int kTmaNumSlots = 2 * 2 * 2 * 2 * kTmaNumCfg * 5;
 static_assert(kTmaNumSlots <= (int)(sizeof(DeviceInfo::tma_max_dyn) / sizeof(size_t)), "opt-in table");
 
-int tma_kernel_slot(int xmode, int cfg, int mt, int rows, int mma) {
+int tma_kernel_slot(int xmode, int cfg, int mt, int rows, int mma, int sf) {
     const int W = kTmaCfg[cfg][0];
     const int mti = mt == 1 ? 0 : (mt == 2 ? 1 : (mt == 4 ? 2 : (mt == 8 ? 3 : (mt == 16 ? 4 : -1))));
     if (mti < 0 || (mt > 1 && (!mma || (W != 8 && W != 16)))) return -1;
-    return (((xmode * 2 + (rows == 16 ? 1 : 0)) * 2 + (mma ? 1 : 0)) * kTmaNumCfg + cfg) * 5 + mti;
+    if (sf && (xmode != 0 || mt != 1 || mma)) return -1;
+    return ((((sf ? 1 : 0) * 2 + xmode) * 2 + (rows == 16 ? 1 : 0)) * 2 + (mma ? 1 : 0)) * kTmaNumCfg * 5 + cfg * 5 + mti;
 }
 
 template <int X, int R, int MM>
@@ -365,22 +367,34 @@ TmaKernel tma_kernel_m(int W, int mt, int mma) {
     return mma ? tma_kernel_w<X, R, 1>(W, mt) : tma_kernel_w<X, R, 0>(W, mt);
 }
 
-TmaKernel tma_kernel_for(int xmode, int cfg, int mt, int rows, int mma) {
-    if (tma_kernel_slot(xmode, cfg, mt, rows, mma) < 0) return nullptr;
+// one int8 token with per-slice staging barriers
+template <int R>
+TmaKernel tma_kernel_sf(int W) {
+    switch (W) {
+        case 4: return gemv_tma_kernel<0, 4, 1, R, 0, 1>;
+        case 8: return gemv_tma_kernel<0, 8, 1, R, 0, 1>;
+        case 12: return gemv_tma_kernel<0, 12, 1, R, 0, 1>;
+        default: return gemv_tma_kernel<0, 16, 1, R, 0, 1>;
+    }
+}
+
+TmaKernel tma_kernel_for(int xmode, int cfg, int mt, int rows, int mma, int sf) {
+    if (tma_kernel_slot(xmode, cfg, mt, rows, mma, sf) < 0) return nullptr;
     const int W = kTmaCfg[cfg][0];
+    if (sf) return rows == 16 ? tma_kernel_sf<16>(W) : tma_kernel_sf<32>(W);
     if (xmode == 0) return rows == 16 ? tma_kernel_m<0, 16>(W, mt, mma) : tma_kernel_m<0, 32>(W, mt, mma);
     return rows == 16 ? tma_kernel_m<1, 16>(W, mt, mma) : tma_kernel_m<1, 32>(W, mt, mma);
 }
 
 // Opts a TMA GEMV variant into the largest dynamic shared memory left beside
 // its static shared memory; returns that size (0 on failure).
-size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int rows, int mma) {
+size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int rows, int mma, int sf) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    const int si = tma_kernel_slot(xmode, cfg, mt, rows, mma);
+    const int si = tma_kernel_slot(xmode, cfg, mt, rows, mma, sf);
     if (si < 0) return 0;
     size_t &slot = dev->tma_max_dyn[si];
     if (slot == 0) {
-        TmaKernel kern = tma_kernel_for(xmode, cfg, mt, rows, mma);
+        TmaKernel kern = tma_kernel_for(xmode, cfg, mt, rows, mma, sf);
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.sharedSizeBytes >= dev->smem_optin) return 0;
         const size_t dyn = dev->smem_optin - fa.sharedSizeBytes;
@@ -470,10 +484,19 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
 int launch_gemv_tma(DeviceInfo *dev, int xmode, const int8_t *q, const uint16_t *x, const uint8_t *packed, int64_t M,
                     int64_t N, int64_t K, int32_t *y_i32, uint16_t *y_bf16, const float *gamma, const float *s_act,
                     const TmaPlan &tp, cudaStream_t st) {
-    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt, tp.rows, tp.mma);
+    // per-slice staging barriers (a variant of its own: one int8 token, dp4a)
+    // where CTAs have many items over few slices; measured on B200: 55296 x
+    // 5120 (120 items per CTA) 13.1 -> 12.3 us; 20480 x 3200 (35) 5.21 ->
+    // 5.13 us alone but the eight-shape sweep 0.15 us slower per step with it;
+    // calls of 15 items or fewer per CTA 0.07-0.19 us slower; 5120 x 27648
+    // (54 slices) 0.2 us slower
+    int sf = (xmode == 0 && tp.mt == 1 && !tp.mma && (int64_t)tp.max_blocks * tp.slices >= 64 && tp.slices <= 32) ? 1 : 0;
+    if (xmode == 0 && tp.mt == 1 && !tp.mma && (gemv_tune().sflags == 0 || gemv_tune().sflags == 1))
+        sf = gemv_tune().sflags;
+    TmaKernel kern = tma_kernel_for(xmode, tp.cfg, tp.mt, tp.rows, tp.mma, sf);
     if (kern == nullptr) return BITNET_ERR_UNSUPPORTED;
     if (tensor_map_encoder() == nullptr ||
-        tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt, tp.rows, tp.mma))
+        tp.smem > tma_max_dynamic_smem(dev, xmode, tp.cfg, tp.mt, tp.rows, tp.mma, sf))
         return BITNET_ERR_CUDA;
     const int64_t row_bytes = packed_row_bytes(K);
     CUtensorMap map;

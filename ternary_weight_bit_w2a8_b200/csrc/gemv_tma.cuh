@@ -79,7 +79,8 @@ __host__ __device__ inline size_t gemv_tma_smem_bytes(int warps, int stages, int
                                                       int tokens = 1, int rows = kTmaRows) {
     return 1024 /* alignment slack */ + (size_t)warps * stages * rows * kTmaSliceBytes +
            (size_t)tokens * gemv_tma_token_stride(slices, tokens) + (size_t)max_blocks_cta * tokens * rows * 4 +
-           (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4;
+           (size_t)max_blocks_cta * 4 + 8 + (size_t)warps * stages * 8 + (size_t)tokens * slices * 4 +
+           (size_t)slices * 8 /* slice barriers (one token, int8) */;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -206,10 +207,12 @@ struct PieceCursor {
 // the sum of every 512-k slice of token t in qslice[t * slices + j].  Piece p
 // (16 k) of the flat (token, piece) order is staged by thread p mod blockDim.x;
 // a warp takes 32 consecutive pieces, one slice of one token, so one warp
-// reduction gives the slice's sum.
+// reduction gives the slice's sum.  With slice_bar (one token), the warp then
+// arrives on slice_bar[j] for each slice j it staged, so that a consumer waits
+// for that slice alone rather than for the whole CTA.
 template <int MT>
 __device__ __forceinline__ void stage_tokens_int8(int8_t *qlin, int64_t ldx, int *qslice, int slices, const int8_t *q,
-                                                  int M, int64_t K, int64_t kq) {
+                                                  int M, int64_t K, int64_t kq, uint64_t *slice_bar = nullptr) {
     PieceCursor<MT> cur((int)(kq / 16));  // ppt and blockDim.x are multiples of 32
     while (cur.valid()) {
         uint4 v[kStageHeld];
@@ -236,6 +239,13 @@ __device__ __forceinline__ void stage_tokens_int8(int8_t *qlin, int64_t ldx, int
             if (ts[i] < MT) {  // warp-uniform
                 *reinterpret_cast<uint4 *>(qlin + ts[i] * ldx + (int64_t)ps[i] * 16) = v[i];
                 slice_sum(qslice + ts[i] * slices, ps[i], v[i]);
+                if (slice_bar != nullptr) {
+                    __syncwarp();  // every lane's piece and the sum are written
+                    if ((threadIdx.x & 31) == 0)
+                        asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(
+                                         smem_u32(&slice_bar[ps[i] >> 5]))
+                                     : "memory");
+                }
             }
         }
     }
@@ -358,10 +368,12 @@ constexpr int gemv_tma_min_blocks() { return MMA ? 1 : ((MT <= 2 || (W <= 8 && M
 //   - Token rows sit ldx = kq + 64 bytes apart, so that the eight tokens' loads
 //     of a quarter warp fall in distinct banks; the box rows' loads are
 //     conflict-free under the 128-byte swizzle (distinct units per row).
-template <int XMODE, int W, int MT, int ROWS, int MMA>
+// SF = 1 (one token, int8, dp4a): per-slice staging barriers (see below).
+template <int XMODE, int W, int MT, int ROWS, int MMA, int SF = 0>
 __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     gemv_tma_kernel(const __grid_constant__ CUtensorMap wmap, const GemvTmaArgs a) {
     static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8 || MT == 16, "tokens per launch");
+    static_assert(SF == 0 || (XMODE == 0 && MT == 1 && MMA == 0), "per-slice barriers: one int8 token, dp4a");
     static_assert(MMA || MT == 1, "several tokens take the MMA path");
     static_assert(ROWS == 32 || ROWS == 16, "rows per box");
     constexpr int kLPR = kTmaRows / ROWS;               // lanes per row (output stores; dp4a MAC)
@@ -392,6 +404,13 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     int *qslice = done + a.max_blocks_cta;                                     // [MT][slices]
     uint64_t *bars =
         reinterpret_cast<uint64_t *>(qslice + MT * slices + ((a.max_blocks_cta + MT * slices) & 1));
+    // one token of int8 activations, launches with many items per CTA: every
+    // 512-k slice is staged by one warp, which arrives on that slice's
+    // barrier, so a warp starts on its items as soon as their slices are in
+    // (no block-wide barrier after the staging; the barriers' set-up costs a
+    // block barrier before the launch-chain wait, which short calls feel)
+    constexpr bool kSliceFlags = SF == 1;
+    uint64_t *slbar = bars + W * ns;  // [slices]
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int brow = lane / kLPR, part = lane % kLPR;  // this lane's box row and chunk half
@@ -441,25 +460,30 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
             issue_next(s);
         }
     }
+    if (kSliceFlags && threadIdx.x == 1) {
+        for (int j = 0; j < slices; ++j) mbar_init(&slbar[j], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     for (int i = threadIdx.x; i < nslots * MT * ROWS; i += blockDim.x) accs[i] = 0;
     for (int i = threadIdx.x; i < nslots; i += blockDim.x) done[i] = 0;
+    if (kSliceFlags) __syncthreads();  // slice barriers and accumulators ready, before the wait
     pdl_launch_dependents();
     pdl_wait();
 
     {
         float sc[MT];
         if (XMODE == 0) {
-            stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq);
+            stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq, kSliceFlags ? slbar : nullptr);
         } else {
             stage_tokens_bf16<MT>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
         }
-        if (threadIdx.x == 0) {
+        if (!kSliceFlags && threadIdx.x == 0) {
 #pragma unroll
             for (int t = 0; t < MT; ++t)
                 fsh[t] = (t < a.M && a.y_bf16 != nullptr) ? __fdiv_rn(*a.gamma, XMODE == 1 ? sc[t] : a.s_act[t]) : 0.0f;
         }
     }
-    __syncthreads();
+    if (!kSliceFlags) __syncthreads();
 
     // dp4a accumulators: one row (or half of one), per code plane
     int acc[4] = {0, 0, 0, 0}, corr = 0;
@@ -521,7 +545,8 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
                 const int tot = atomicAdd(&accs[(sl * MT + t) * ROWS + brow], 0);
                 if (part == 0 && t < a.M && n < a.N) {
                     if (a.y_bf16 != nullptr)
-                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(__fmul_rn((float)tot, fsh[t]));
+                        a.y_bf16[(int64_t)t * a.N + n] = float_to_bf16_bits_rn(
+                            __fmul_rn((float)tot, kSliceFlags ? __fdiv_rn(*a.gamma, a.s_act[0]) : fsh[t]));
                     else
                         a.y_i32[(int64_t)t * a.N + n] = tot;
                 }
@@ -536,6 +561,13 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
     int s = 0;
     uint32_t phase = 0;
     for (int n = 0; n < n_items; ++n) {
+        if (kSliceFlags && !mbar_wait_bounded(&slbar[cj], 0u)) {
+            if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
+            // wait (bounded) for this warp's boxes in flight, then stop
+            for (int d = 0; d < ns && n + d < n_items; ++d)
+                mbar_wait_bounded(&mybar[(n + d) % ns], (uint32_t)((n + d) / ns) & 1u);
+            break;
+        }
         if (!mbar_wait_bounded(&mybar[s], phase)) {
             if (lane == 0) record_device_error(BITNET_ERR_DEVICE_TIMEOUT);
             // wait (bounded) for this warp's other boxes still in flight, then stop

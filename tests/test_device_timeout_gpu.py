@@ -41,7 +41,8 @@ print(json.dumps({"status": status, "again": again, "exact_after": exact, "secon
 """
 
 
-@pytest.mark.parametrize("tune", [None, "0,0,0,0,-1,0,3"])  # the planner's variant; 16 warps
+# the planner's variant; 16 warps; per-slice staging barriers
+@pytest.mark.parametrize("tune", [None, "0,0,0,0,-1,0,3", "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,-1,1"])
 def test_bounded_wait_reports_timeout_and_context_survives(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():

@@ -59,11 +59,12 @@ print(json.dumps(out))
 """
 
 
-# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma,l2":
+# BITNET_GEMV_TUNE = "G,R,U,ctas_per_sm,prefetch,S,variant,ring,fuse,qwpt,rows,cores,mma,l2,sflags":
 # variant 1..5 = 8x4, 12x3, 16x2, 8x2, 4x4 (warps x most boxes per warp), rows
 # per block 16 or 32, cores = 1 the co-residency mode (two CTAs per SM), mma =
 # 1 / 0 the MMA or the dp4a product for one token, l2 = 0 weights without the
-# L2 evict-first policy.  4832 x 27648 and 20000 x
+# L2 evict-first policy, sflags = 1 / 0 per-slice staging barriers always /
+# never.  4832 x 27648 and 20000 x
 # 3200 leave 3 and 136 CTAs with one 32-row block more than the others.
 @pytest.mark.parametrize("tune", ["0,0,0,0,-1,0,-1",     # the planner's own choice
                                   "0,0,0,0,-1,0,1",      # 8 warps, ring up to 4
@@ -79,7 +80,10 @@ print(json.dumps(out))
                                   "0,0,0,0,-1,0,1,0,-1,0,16,-1,1",  # MMA, 16-row blocks, 8 warps
                                   "0,0,0,0,-1,0,2,0,-1,0,0,-1,1",  # MMA, 12 warps
                                   "0,0,0,0,-1,0,-1,0,-1,0,0,-1,0",  # dp4a product for one token
-                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,0"])  # weights without the evict-first policy
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,0",  # weights without the evict-first policy
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,-1,1",  # per-slice staging barriers always
+                                  "0,0,0,0,-1,0,5,0,-1,0,16,-1,-1,-1,1",  # the same, 4 warps, 16-row blocks
+                                  "0,0,0,0,-1,0,-1,0,-1,0,0,-1,-1,-1,0"])  # never
 def test_tma_path_forced_small_shapes(tune):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
