@@ -160,6 +160,56 @@ def replay_steps(graphs, n, multi=None):
         graphs[j % C].replay()
 
 
+HOLD_CYCLES = 4_000_000  # ~2 ms of device spinning before a timed region
+
+
+def step_plan(steps, chunk):
+    """How `timed_steps` covers exactly `steps` steps: [(first step, steps in
+    the graph, replays)], a graph of `chunk` steps replayed while whole chunks
+    remain, then one graph of the remainder."""
+    n_big, rem = divmod(steps, chunk)
+    plan = []
+    if n_big:
+        plan.append((0, chunk, n_big))
+    if rem:
+        plan.append((n_big * chunk, rem, 1))
+    return plan
+
+
+def timed_steps(torch, step_fn, steps, warmup, dist=None, chunk=448):
+    """Times exactly `steps` steps: `step_fn(i0, n)` enqueues steps i0 .. i0 +
+    n - 1 (step i decides its own rotation copy, so `chunk` is a multiple of
+    the copy count).  The timed sequence is captured as at most two CUDA graphs
+    (see step_plan), each replayed once beforehand, so that graph boundaries
+    (a few us each) do not depend on the run length; `warmup` steps run
+    untimed first.  Returns the elapsed ms (max over ranks)."""
+    graphs = [(capture(torch, lambda i0=i0, n=n: step_fn(i0, n)), r) for (i0, n, r) in step_plan(steps, chunk)]
+    for g, _ in graphs:
+        g.replay()
+    if warmup:
+        step_fn(0, warmup)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    hold = getattr(torch.cuda, "_sleep", None)
+    if hold is not None:
+        hold(HOLD_CYCLES)
+    start.record()
+    for g, r in graphs:
+        for _ in range(r):
+            g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(torch, start.elapsed_time(end), dist, "cuda")
+    if dist is not None:
+        dist.barrier()
+    del graphs
+    return ms
+
+
 def timed_graph_loop(torch, graphs, steps, warmup, dist=None, multi=None):
     """Every graph replayed once (so the first replay's one-time cost never
     lands in the timed region, whatever `warmup` is), `warmup` untimed steps,
@@ -176,6 +226,13 @@ def timed_graph_loop(torch, graphs, steps, warmup, dist=None, multi=None):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    # keep the GPU busy (outside the timed region) while the host enqueues the
+    # timed graphs, so that the start event is not followed by a wait for the
+    # first submission: short runs then time the same back-to-back steps as
+    # long ones
+    hold = getattr(torch.cuda, "_sleep", None)
+    if hold is not None:
+        hold(HOLD_CYCLES)
     start.record()
     replay_steps(graphs, steps, multi)
     end.record()
@@ -248,18 +305,22 @@ class GemvSet:
 
 def measure_gemv_set(torch, bn, gs, steps, warmup, dist=None, clocks=None):
     """Headline: a step is the calls of all shapes back to back (linked by
-    programmatic dependent launch) over one rotation copy.  One graph holds the
-    steps of all copies in turn and is replayed whole; single-step graphs run
-    the remainder, so exactly `steps` steps are timed."""
+    programmatic dependent launch) over one rotation copy, step i on copy i mod
+    C.  Exactly `steps` steps are timed, captured in graphs of 64 rounds of the
+    copies (see timed_steps)."""
+    C = len(gs.copies)
     n_before = bn.bitnet_launch_count()
-    graphs = [capture(torch, lambda c=c: gs.run(c)) for c in range(len(gs.copies))]
-    launches_per_step = (bn.bitnet_launch_count() - n_before) // (2 * len(gs.copies))
-    multi = capture(torch, lambda: [gs.run(c) for c in range(len(gs.copies))])
+    gs.run(0)
+    torch.cuda.synchronize()
+    launches_per_step = bn.bitnet_launch_count() - n_before
+
+    def step_fn(i0, n):
+        for i in range(i0, i0 + n):
+            gs.run(i % C)
     if clocks is not None:
         clocks.start()
-    ms = timed_graph_loop(torch, graphs, steps, warmup, dist, multi)
+    ms = timed_steps(torch, step_fn, steps, warmup, dist, chunk=64 * C)
     clk = clocks.stop() if clocks is not None else None
-    del graphs, multi
     return ms, launches_per_step, clk
 
 
@@ -271,13 +332,13 @@ def per_launch_us(torch, bn, gs, warmup, reps=30):
     C = len(gs.copies)
     for j, (N, K) in enumerate(gs.shapes):
         L = 4 * C
-        def run(j=j, N=N, L=L):
-            for i in range(L):
-                bn.bitnet_w2a8_gemm(gs.q[j], gs.copies[i % C][j], N, y=gs.y[j], ws=gs.ws[j])
-        g = capture(torch, run)
-        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+
+        def step_fn(i0, n, j=j, N=N, L=L):  # a step: L back-to-back calls
+            for _ in range(n):
+                for i in range(L):
+                    bn.bitnet_w2a8_gemm(gs.q[j], gs.copies[i % C][j], N, y=gs.y[j], ws=gs.ws[j])
+        ms = timed_steps(torch, step_fn, reps, max(3, warmup // 10), chunk=reps)
         out.append(ms * 1e3 / (reps * L))
-        del g
     return out
 
 

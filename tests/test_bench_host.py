@@ -130,3 +130,14 @@ def test_traffic_hash_covers_the_gemv_not_the_tensor_core_gemm(tmp_path, monkeyp
     (dst / "gemv_tma.cuh").write_text((dst / "gemv_tma.cuh").read_text(encoding="utf-8") + "\n// edit\n",
                                       encoding="utf-8")
     assert bench.kernel_source_hash() != h0          # a GEMV edit invalidates it
+
+
+def test_step_plan_covers_exactly_the_steps():
+    for steps in (1, 5, 20, 447, 448, 449, 896, 20000):
+        plan = bench.step_plan(steps, 448)
+        assert len(plan) <= 2
+        assert sum(n * r for (_, n, r) in plan) == steps
+        i = 0
+        for (i0, n, r) in plan:  # graphs in order, each starting where the last left off
+            assert i0 == i and i0 % 7 == 0
+            i += n * r
