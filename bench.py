@@ -147,19 +147,6 @@ def job_gbps(bytes_per_step_per_rank, steps, ms_max, world):
     return world * bytes_per_step_per_rank * steps / (ms_max * 1e-3) / 1e9
 
 
-def replay_steps(graphs, n, multi=None):
-    """Runs exactly `n` steps: `graphs[c]` is one step over rotation copy c;
-    `multi` (optional) holds all len(graphs) steps, copy 0 first, in one graph."""
-    C = len(graphs)
-    i = 0
-    if multi is not None:
-        for _ in range(n // C):
-            multi.replay()
-        i = (n // C) * C
-    for j in range(i, n):
-        graphs[j % C].replay()
-
-
 HOLD_CYCLES = 4_000_000  # ~2 ms of device spinning before a timed region
 
 
@@ -207,39 +194,6 @@ def timed_steps(torch, step_fn, steps, warmup, dist=None, chunk=448):
     if dist is not None:
         dist.barrier()
     del graphs
-    return ms
-
-
-def timed_graph_loop(torch, graphs, steps, warmup, dist=None, multi=None):
-    """Every graph replayed once (so the first replay's one-time cost never
-    lands in the timed region, whatever `warmup` is), `warmup` untimed steps,
-    then exactly `steps` timed ones (see replay_steps).  Returns the elapsed ms
-    (max over ranks)."""
-    if multi is not None:
-        multi.replay()
-    for g in graphs:
-        g.replay()
-    replay_steps(graphs, warmup, multi)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    # keep the GPU busy (outside the timed region) while the host enqueues the
-    # timed graphs, so that the start event is not followed by a wait for the
-    # first submission: short runs then time the same back-to-back steps as
-    # long ones
-    hold = getattr(torch.cuda, "_sleep", None)
-    if hold is not None:
-        hold(HOLD_CYCLES)
-    start.record()
-    replay_steps(graphs, steps, multi)
-    end.record()
-    torch.cuda.synchronize()
-    ms = max_over_ranks(torch, start.elapsed_time(end), dist, "cuda")
-    if dist is not None:
-        dist.barrier()
     return ms
 
 
@@ -438,12 +392,12 @@ def measure_bitlinear_decode(torch, bn, shapes, warmup, l2_bytes, reps=30):
         def run():
             for i in range(L):
                 bn.bitnet_bitlinear(xd, copies[i % C], gamma, N, y=y, ws=ws)
-        g = capture(torch, run)
-        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+        ms = timed_steps(torch, lambda i0, n, f=run: [f() for _ in range(n)], reps,
+                         max(3, warmup // 10), chunk=reps)
         us = ms * 1e3 / (reps * L)
         out.append({"N": N, "K": K, "us_per_call": round(us, 3),
                     "GBps": round(bitlinear_bytes(1, N, K) / (us * 1e-6) / 1e9, 1)})
-        del g, copies
+        del copies
     return out
 
 
@@ -474,13 +428,12 @@ def measure_small_batch(torch, bn, shapes, ms_list, warmup, l2_bytes, reps=30):
                 def run(fn=fn):
                     for i in range(L):
                         fn(i)
-                g = capture(torch, run)
-                ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+                ms = timed_steps(torch, lambda i0, n, f=run: [f() for _ in range(n)], reps,
+                                 max(3, warmup // 10), chunk=reps)
                 us = ms * 1e3 / (reps * L)
                 nbytes = gemv_bytes(M, N, K) if name == "int32" else bitlinear_bytes(M, N, K)
                 row[f"{name}_us_per_call"] = round(us, 3)
                 row[f"{name}_GBps"] = round(nbytes / (us * 1e-6) / 1e9, 1)
-                del g
             out.append(row)
         del copies
     return out
@@ -507,21 +460,19 @@ def measure_prefill(torch, bn, ms_list, shapes, warmup, int8_peak_tops, reps=20,
             def run():
                 for _ in range(L):
                     bn.bitnet_w2a8_gemm(q, packed, N, y=y, ws=ws)
-            g = capture(torch, run)
-            ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+            ms = timed_steps(torch, lambda i0, n, f=run: [f() for _ in range(n)], reps,
+                             max(3, warmup // 10), chunk=reps)
             us = ms * 1e3 / (reps * L)
             tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
-            del g
             yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
             wsb = bn.workspace(M, N, K)
 
             def run_bl():
                 for _ in range(L):
                     bn.bitnet_bitlinear(xd, packed, gamma, N, y=yb, ws=wsb)
-            g = capture(torch, run_bl)
-            ms_bl = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+            ms_bl = timed_steps(torch, lambda i0, n, f=run_bl: [f() for _ in range(n)], reps,
+                             max(3, warmup // 10), chunk=reps)
             us_bl = ms_bl * 1e3 / (reps * L)
-            del g
             out.append({"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "int8_TOPS": round(tops, 1),
                         "frac_int8_peak": round(tops / int8_peak_tops, 4),
                         "GBps": round(gemv_bytes(M, N, K) / (us * 1e-6) / 1e9, 1),
@@ -546,12 +497,12 @@ def measure_bf16_context(torch, shapes, warmup, l2_bytes, reps=30):
         def run():
             for i in range(L):
                 torch.matmul(x, ws[i % C], out=y)
-        g = capture(torch, run)
-        ms = timed_graph_loop(torch, [g], reps, max(3, warmup // 10))
+        ms = timed_steps(torch, lambda i0, n, f=run: [f() for _ in range(n)], reps,
+                         max(3, warmup // 10), chunk=reps)
         us = ms * 1e3 / (reps * L)
         out.append({"N": N, "K": K, "bf16_us_per_call": round(us, 3),
                     "GBps": round((2 * N * K + 2 * K + 2 * N) / (us * 1e-6) / 1e9, 1)})
-        del g, ws
+        del ws
         torch.cuda.empty_cache()
     return out
 

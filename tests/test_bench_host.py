@@ -96,24 +96,6 @@ def test_traffic_valid_only_for_the_captured_sources(tmp_path):
     assert bench.read_traffic(str(tmp_path / "missing.json")) is None
 
 
-def test_replay_steps_runs_exactly_n_steps():
-    class G:
-        def __init__(self, log, tag):
-            self.log, self.tag = log, tag
-
-        def replay(self):
-            self.log.append(self.tag)
-
-    for n in (0, 1, 6, 7, 15, 20):
-        log = []
-        singles = [G(log, (c,)) for c in range(7)]
-        multi = G(log, tuple(range(7)))
-        bench.replay_steps(singles, n, multi)
-        steps = [c for t in log for c in t]
-        assert len(steps) == n
-        assert steps == [i % 7 for i in range(n)]  # every step on the next rotation copy
-
-
 def test_traffic_hash_covers_the_gemv_not_the_tensor_core_gemm(tmp_path, monkeypatch):
     import shutil
     src = os.path.join(ROOT, "ternary_weight_bit_w2a8_b200", "csrc")
