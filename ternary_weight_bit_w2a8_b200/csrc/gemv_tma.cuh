@@ -257,12 +257,13 @@ __device__ __forceinline__ void stage_tokens_int8(int8_t *qlin, int64_t ldx, int
 // together), one block reduction for all tokens, then the codes, with slice
 // sums as above.  Pieces beyond those held are read again.  Returns the
 // scales in sc; token slots t >= M are staged as zeros.  `red` holds MT x 32
-// floats.
-template <int MT>
+// floats; NW is the CTA's warp count (the per-warp maxima are read back with
+// all loads in flight at once).
+template <int MT, int NW>
 __device__ __forceinline__ void stage_tokens_bf16(int8_t *qlin, int64_t ldx, int *qslice, int slices, float *red,
                                                   const uint16_t *x, int M, int64_t K, int64_t kq, float (&sc)[MT]) {
     const int ppt = (int)(kq / 16);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     auto load = [&](int t, int pp, uint4 &lo, uint4 &hi) {
         lo = hi = make_uint4(0u, 0u, 0u, 0u);
         if (t < M) {
@@ -306,7 +307,8 @@ __device__ __forceinline__ void stage_tokens_bf16(int8_t *qlin, int64_t ldx, int
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         float v = 0.0f;
-        for (int w = 0; w < nwarps; ++w) v = fmaxf(v, red[t * 32 + w]);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) v = fmaxf(v, red[t * 32 + w]);
         sc[t] = t < M ? __fdiv_rn(127.0f, v > kQuantEps ? v : kQuantEps) : 0.0f;
     }
     auto put = [&](int t, int pp, const uint4 &lo, const uint4 &hi) {  // t < MT: warp-uniform
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(W * 32, gemv_tma_min_blocks<W, MT, MMA>())
         if (XMODE == 0) {
             stage_tokens_int8<MT>(qlin, ldx, qslice, slices, a.q, a.M, a.K, kq, kSliceFlags ? slbar : nullptr);
         } else {
-            stage_tokens_bf16<MT>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
+            stage_tokens_bf16<MT, W>(qlin, ldx, qslice, slices, red, a.x, a.M, a.K, kq, sc);
         }
         if (!kSliceFlags && threadIdx.x == 0) {
 #pragma unroll
