@@ -578,11 +578,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int64_t n0 = (int64_t)t.nt * kTcRows, m0 = (int64_t)t.mt * BT;
             const int64_t n = n0 + row;
             const uint32_t dt = tq + (uint32_t)(d * BT);
-            // BitLinear factor gamma / s_m of token c0 + lane (lanes share it by shuffle)
-            auto token_factor = [&](int c0) {
-                const int64_t m = m0 + c0 + lane;
-                return (BF16_OUT && m < a.M) ? __fdiv_rn(*a.gamma, a.s_act[m]) : 0.0f;
-            };
+            // BitLinear factors gamma / s_m of the unit's tokens: a table per
+            // epilogue warp in the upper half of its first staging buffer (bf16
+            // boxes fill only the lower 2 KB), read back four at a time
+            float *fac = reinterpret_cast<float *>(wbuf + 2048);
+            if (BF16_OUT) {
+                for (int c = lane; c < BT; c += 32) {
+                    const int64_t m = m0 + c;
+                    fac[c] = m < a.M ? __fdiv_rn(*a.gamma, a.s_act[m]) : 0.0f;
+                }
+                __syncwarp();
+            }
             uint32_t v[16];
             if (a.tma_store) {
                 // boxes of (up to) 32 tokens x 32 weight rows, row-major by token as y is
@@ -593,16 +599,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (lane == 0) tma_store_wait_read<kTcEpiBufs - 1>();
                         __syncwarp();
                     }
-                    const float fl = token_factor(c0);
 #pragma unroll
                     for (int h = 0; h < kTok / 16; ++h) {
                         tmem_ld16(dt + (uint32_t)(c0 + 16 * h), v);
+                        float f[16];
+                        if (BF16_OUT) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 f4 = reinterpret_cast<const float4 *>(fac + c0 + 16 * h)[i];
+                                f[4 * i] = f4.x, f[4 * i + 1] = f4.y, f[4 * i + 2] = f4.z, f[4 * i + 3] = f4.w;
+                            }
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int tk = 16 * h + i;
                             if (BF16_OUT)
-                                reinterpret_cast<uint16_t *>(buf)[tk * 32 + lane] = float_to_bf16_bits_rn(
-                                    __fmul_rn((float)(int)v[i], __shfl_sync(0xffffffffu, fl, tk)));
+                                reinterpret_cast<uint16_t *>(buf)[tk * 32 + lane] =
+                                    float_to_bf16_bits_rn(__fmul_rn((float)(int)v[i], f[i]));
                             else
                                 reinterpret_cast<uint32_t *>(buf)[tk * 32 + lane] = v[i];
                         }
@@ -620,10 +633,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
                 for (int c0 = 0; c0 < BT; c0 += 16) {
                     tmem_ld16(dt + (uint32_t)c0, v);
-                    const float fl = token_factor(c0);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float f = __shfl_sync(0xffffffffu, fl, i);
+                        const float f = BF16_OUT ? fac[c0 + i] : 0.0f;
                         const int64_t m = m0 + c0 + i;
                         if (n < a.N && m < a.M) {
                             if (BF16_OUT)
