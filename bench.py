@@ -147,9 +147,6 @@ def job_gbps(bytes_per_step_per_rank, steps, ms_max, world):
     return world * bytes_per_step_per_rank * steps / (ms_max * 1e-3) / 1e9
 
 
-HOLD_CYCLES = 4_000_000  # ~2 ms of device spinning before a timed region
-
-
 def step_plan(steps, chunk):
     """How `timed_steps` covers exactly `steps` steps: [(first step, steps in
     the graph, replays)], a graph of `chunk` steps replayed while whole chunks
@@ -181,9 +178,6 @@ def timed_steps(torch, step_fn, steps, warmup, dist=None, chunk=448):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    hold = getattr(torch.cuda, "_sleep", None)
-    if hold is not None:
-        hold(HOLD_CYCLES)
     start.record()
     for g, r in graphs:
         for _ in range(r):
