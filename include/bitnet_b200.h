@@ -142,7 +142,7 @@ BITNET_API int bitnet_quant_act(const uint16_t *x, int64_t M, int64_t K, int8_t 
  * int8 activations with the ternary weights, equal element by element to an
  * integer matmul):
  *   y[m,n] = sum_k q[m,k] * W_t[n,k]    exact in int32.
- * Paths: M <= 8 with K >= 512 runs the TMA-staged GEMV, one pass over the
+ * Paths: M <= 16 with K >= 512 runs the TMA-staged GEMV, one pass over the
  * weights for all M tokens; M >= 2 otherwise (K >= 128) runs the persistent
  * tcgen05 tensor-core GEMM; what remains (M == 1 with K < 512, or K < 128)
  * runs the register-streaming GEMV.  All give the same exact result.
