@@ -157,11 +157,18 @@ int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_
     while (wpt < 8 && ceil_div(K, 8) > (int64_t)kQuantHeld * 32 * wpt) wpt *= 2;
     const int tw = gemv_tune().qwpt;
     if (tw == 1 || tw == 2 || tw == 4 || tw == 8) wpt = tw;
-    const int64_t teams_per_cta = kThreads / (32 * wpt);
+    // teams per CTA: up to kThreads / (32 wpt), fewer when that spreads one
+    // wave of tokens over every SM (2048 tokens: 147 CTAs of 14 one-warp
+    // teams rather than 128 of 16)
+    int64_t teams_per_cta = kThreads / (32 * wpt);
+    if (M <= (int64_t)dev->sm_count * teams_per_cta) {
+        const int64_t t = ceil_div(M, (int64_t)dev->sm_count);
+        if (t >= 1 && t < teams_per_cta) teams_per_cta = t;
+    }
     int64_t grid = ceil_div(M, teams_per_cta);
     const int64_t cap = (int64_t)dev->sm_count * (2048 / kThreads);
     if (grid > cap) grid = cap;
-    const dim3 g((unsigned)grid), b(kThreads);
+    const dim3 g((unsigned)grid), b((unsigned)(teams_per_cta * 32 * wpt));
     cudaError_t e;
     switch (wpt) {
         case 1: e = launch_pdl(quant_act_kernel<1>, g, b, 0, st, x, M, K, q, ldq, zero_pad, s, rowsum); break;
@@ -453,9 +460,17 @@ TmaPlan tma_plan(int64_t M, int64_t N, int64_t K) {
     // the second lane of a row
     const bool cores = tn.cores == 1;
     p.rows = (!cores || ceil_div(N, kTmaRows) >= kRefSMs || p.mt >= 8) ? 32 : 16;
+    p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
+    // long rows (>= 32 slices) with a leftover of 32-row blocks: 16-row blocks
+    // where they cut the busiest CTA's rows by a fifth (5120 x 27648: 64 -> 48
+    // rows, 11.2 -> 10.7 us on B200; shorter rows measured slower with them)
+    if (!cores && p.mt == 1 && p.slices >= 32) {
+        const int64_t r32 = ceil_div(ceil_div(N, 32), (int64_t)kRefSMs) * 32;
+        const int64_t r16 = ceil_div(ceil_div(N, 16), (int64_t)kRefSMs) * 16;
+        if (r16 * 5 <= r32 * 4) p.rows = 16;
+    }
     if (tn.rows == 16 || tn.rows == 32) p.rows = tn.rows;
     p.nblocks = ceil_div(N, p.rows);
-    p.slices = (int)ceil_div(row_bytes, kTmaSliceBytes);
     if (tune >= 1 && tune <= kTmaNumCfg)
         p.cfg = tune - 1;
     else

@@ -72,8 +72,8 @@ __device__ __forceinline__ uint2 quant8(const uint4 &v, float sc, int &sum) {
     return make_uint2(pack4_b0(c[0], c[1], c[2], c[3]), pack4_b0(c[4], c[5], c[6], c[7]));
 }
 
-// A team of WPT warps quantises one token row at a time (a CTA of kThreads
-// threads holds kThreads / (32 * WPT) teams; rows are dealt to teams
+// A team of WPT warps quantises one token row at a time (a CTA of up to
+// kThreads threads holds blockDim.x / (32 * WPT) teams; rows are dealt to teams
 // grid-stride).  The row is read from HBM once: each thread keeps up to
 // kQuantHeld 16-byte words in registers between the absmax pass and the
 // quantise pass (rows longer than kQuantHeld * 8 * 32 * WPT values re-read
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t *__r
                                                              int8_t *__restrict__ q, int64_t ldq, bool zero_pad,
                                                              float *__restrict__ s, int32_t *__restrict__ rowsum) {
     constexpr int kTeam = 32 * WPT;
-    constexpr int kTeams = kThreads / kTeam;
+    const int teams = blockDim.x / kTeam;  // blockDim.x: a multiple of kTeam, at most kThreads
     __shared__ float fred[kThreads / 32];
     __shared__ int ired[kThreads / 32];
     // a dependent kernel may start its own independent work (weight loads)
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t *__r
     pdl_launch_dependents();
     pdl_wait();
     const int team = threadIdx.x / kTeam, t = threadIdx.x % kTeam;
-    for (int64_t m = (int64_t)blockIdx.x * kTeams + team; m < M; m += (int64_t)gridDim.x * kTeams) {
+    for (int64_t m = (int64_t)blockIdx.x * teams + team; m < M; m += (int64_t)gridDim.x * teams) {
         int sum = 0;
         const float sc = quant_row<WPT>(x + m * K, K, q + m * ldq, ldq, zero_pad, rowsum != nullptr, sum, fred, ired,
                                         team, t);
