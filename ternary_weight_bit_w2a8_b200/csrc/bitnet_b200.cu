@@ -414,11 +414,13 @@ size_t tma_max_dynamic_smem(DeviceInfo *dev, int xmode, int cfg, int mt, int row
 // Plan of the TMA GEMV, from the shape and B200 reference figures only (148
 // SMs, 228 KB of shared memory per SM), so that what a shape needs does not
 // depend on the device that runs it.
-//   - Row blocks of 32 rows; CTA c takes row blocks c, c + grid, ..., with at
-//     most 148 CTAs.
+//   - Row blocks of 32 rows (16 for long rows where that evens out the
+//     busiest CTA, see below); CTA c takes row blocks c, c + grid, ..., with
+//     at most 148 CTAs.
 //   - Variant (measured on B200): 16 warps x up to 2 boxes in flight, 12 x 3
-//     for rows of >= 32 K-slices; 8 or 16 warps for several tokens.  The ring
-//     is no deeper than the warp's items need.
+//     for rows of >= 32 K-slices; 8 or 16 warps for several tokens (the MMA
+//     product, up to 16 tokens).  The ring is no deeper than the warp's items
+//     need.
 //   - One CTA per SM per launch, for every launch: its shared memory is padded
 //     past half an SM.  Programmatic dependent launch could otherwise start
 //     the next call's CTAs beside this call's, to request their weights early;
