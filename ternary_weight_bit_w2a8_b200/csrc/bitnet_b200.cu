@@ -158,8 +158,8 @@ int launch_quant(DeviceInfo *dev, const uint16_t *x, int64_t M, int64_t K, int8_
     const int tw = gemv_tune().qwpt;
     if (tw == 1 || tw == 2 || tw == 4 || tw == 8) wpt = tw;
     // teams per CTA: up to kThreads / (32 wpt), fewer when that spreads one
-    // wave of tokens over every SM (2048 tokens: 147 CTAs of 14 one-warp
-    // teams rather than 128 of 16)
+    // wave of tokens over every SM (1024 tokens: 147 CTAs of 7 one-warp teams
+    // rather than 128 of 8)
     int64_t teams_per_cta = kThreads / (32 * wpt);
     if (M <= (int64_t)dev->sm_count * teams_per_cta) {
         const int64_t t = ceil_div(M, (int64_t)dev->sm_count);
