@@ -62,6 +62,16 @@ def test_workspace_bytes(lib):
     assert lib.bitnet_workspace_bytes(3, 100, 1000) == lib.bitnet_workspace_bytes(3, 100, 1000)
 
 
+def test_workspace_bytes_cover_the_bitlinear_quantisation(lib):
+    # 5..16 tokens: BitLinear quantises them into the workspace (q, then the
+    # scales) before the one-pass GEMV
+    for M in (5, 8, 12, 16):
+        assert lib.bitnet_workspace_bytes(M, 300, 2560) >= M * 2560 + M * 4
+    # prefill: K_pad-strided q and the scales ahead of the tensor-core GEMM
+    assert lib.bitnet_workspace_bytes(128, 13824, 2560) >= 128 * 2560 + 128 * 4
+    assert lib.bitnet_workspace_bytes(2048, 2560, 6912) >= 2048 * 6912 + 2048 * 4
+
+
 # The tests below pass fake pointers; each call is built to fail a host-side
 # check before any device work.  They are skipped where a GPU is present, so
 # that a wrong expectation can never turn into a launch on fake pointers.
